@@ -1,0 +1,297 @@
+"""Pins of the oracle's attention and cache model against things other than itself:
+brute-force full-sequence masked attention (pure Python loops), a torch float64 SDPA
+witness, closed forms, softmax row sums, R-way splits, and the ring's closed form."""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from kv_cache_serving_ws_b200 import synth
+from oracle import ws_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _cfg(**kw):
+    base = dict(n_layers=2, n_heads=2, head_dim=4, n_video=3, n_audio=1, n_cond=2, history_units=2)
+    base.update(kw)
+    return orc.Config(**base)
+
+
+def _bits(seed, kind, shape, unit=0, layer=0, step=0):
+    return synth.normal_tensor(synth.stream_key(seed, kind, unit, layer, step), shape)
+
+
+def _fill(cache, cfg, units, seed=1, commit=True, skip_latent=()):
+    """Append COND for every unit, and commit latents for all but the last (and not those in skip_latent)."""
+    for u in units:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        assert cache.append(u, orc.SEG_COND, _bits(seed, synth.KIND_COND_K, cs, u),
+                            _bits(seed, synth.KIND_COND_V, cs, u)) == orc.OK
+        if commit and u != units[-1] and u not in skip_latent:
+            ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+            assert cache.append(u, orc.SEG_LATENT, _bits(seed, synth.KIND_COMMIT_K, ls, u),
+                                _bits(seed, synth.KIND_COMMIT_V, ls, u)) == orc.OK
+
+
+# ------------------------------------------------------------ brute force --
+
+def _brute_force(cfg, seq, q_unit, layer, q_rows):
+    """Full-sequence attention by the definition, with pure-Python loops.
+
+    seq: list of (unit, kind, k[D]..., v[D]...) for every token of every unit in
+    arrival order, kind in {"cond", "latent"}.  The dense block-causal mask is
+    M[i, j] = u(j) <= u(i) and u(j) >= u(i) - U.  Query rows are the latent tokens
+    of q_unit.  Returns out[row][head][d].
+    """
+    U = cfg.history_units
+    D = cfg.head_dim
+    out = []
+    for qi in q_rows:                             # qi: per-head query vectors of one latent token
+        row = []
+        for h in range(cfg.n_heads):
+            logits, vals = [], []
+            for (u, _kind, kvec, vvec) in seq:
+                if u <= q_unit and u >= q_unit - U:
+                    s = sum(qi[h][d] * kvec[h][d] for d in range(D)) / math.sqrt(D)
+                    logits.append(s)
+                    vals.append(vvec[h])
+            m = max(logits)
+            w = [math.exp(s - m) for s in logits]
+            z = sum(w)
+            row.append([sum(w[j] * vals[j][d] for j in range(len(w))) / z for d in range(D)])
+        out.append(row)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("U,units,q_unit_layer", [(2, [0, 1, 2, 3, 4], 1), (1, [0, 1, 2], 0),
+                                                   (3, [0, 1], 1), (0, [5, 6], 0), (2, [0, 1, 3, 4], 1)])
+def test_incremental_equals_full_recomputation(U, units, q_unit_layer):
+    cfg = _cfg(history_units=U)
+    cache = orc.UnitCache(cfg)
+    _fill(cache, cfg, units)
+    u = units[-1]
+    layer = q_unit_layer
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q = _bits(1, synth.KIND_Q, qs, u, layer)
+    kn = _bits(1, synth.KIND_K_NEW, qs, u, layer)
+    vn = _bits(1, synth.KIND_V_NEW, qs, u, layer)
+    st, out = cache.unit_attention(layer, u, q, kn, vn)
+    assert st == orc.OK
+
+    # independent full sequence: every unit's tokens, in arrival order
+    seq = []
+    for uu in units:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        ck = orc.bf16_to_f64(_bits(1, synth.KIND_COND_K, cs, uu))[layer]
+        cv = orc.bf16_to_f64(_bits(1, synth.KIND_COND_V, cs, uu))[layer]
+        seq += [(uu, "cond", ck[t], cv[t]) for t in range(cfg.n_cond)]
+        if uu == u:
+            lk, lv = orc.bf16_to_f64(kn), orc.bf16_to_f64(vn)
+        else:
+            ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+            lk = orc.bf16_to_f64(_bits(1, synth.KIND_COMMIT_K, ls, uu))[layer]
+            lv = orc.bf16_to_f64(_bits(1, synth.KIND_COMMIT_V, ls, uu))[layer]
+        seq += [(uu, "latent", lk[t], lv[t]) for t in range(cfg.n_query)]
+    want = _brute_force(cfg, seq, u, layer, orc.bf16_to_f64(q))
+    assert np.max(np.abs(out - want)) <= 1e-12
+
+
+def test_torch_sdpa_witness_float64():
+    cfg = _cfg(n_heads=3, head_dim=8, n_video=5, n_audio=2, n_cond=3, history_units=2)
+    cache = orc.UnitCache(cfg)
+    units = [0, 1, 2, 3]
+    _fill(cache, cfg, units, seed=9)
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q = _bits(9, synth.KIND_Q, qs, 3)
+    kn = _bits(9, synth.KIND_K_NEW, qs, 3)
+    vn = _bits(9, synth.KIND_V_NEW, qs, 3)
+    st, out = cache.unit_attention(0, 3, q, kn, vn)
+    assert st == orc.OK
+    # build the full sequence (including unit 0, which the mask must hide) and mask it in torch
+    ks, vs, owner = [], [], []
+    for uu in units:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        ks.append(orc.bf16_to_f64(_bits(9, synth.KIND_COND_K, cs, uu))[0])
+        vs.append(orc.bf16_to_f64(_bits(9, synth.KIND_COND_V, cs, uu))[0])
+        owner += [uu] * cfg.n_cond
+        if uu == 3:
+            ks.append(orc.bf16_to_f64(kn)); vs.append(orc.bf16_to_f64(vn))
+        else:
+            ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+            ks.append(orc.bf16_to_f64(_bits(9, synth.KIND_COMMIT_K, ls, uu))[0])
+            vs.append(orc.bf16_to_f64(_bits(9, synth.KIND_COMMIT_V, ls, uu))[0])
+        owner += [uu] * cfg.n_query
+    K = torch.from_numpy(np.concatenate(ks)).permute(1, 0, 2)      # [H, Nk, D]
+    V = torch.from_numpy(np.concatenate(vs)).permute(1, 0, 2)
+    Q = torch.from_numpy(orc.bf16_to_f64(q)).permute(1, 0, 2)      # [H, Nq, D]
+    owner = torch.tensor(owner)
+    mask = (owner <= 3) & (owner >= 3 - cfg.history_units)
+    mask = mask[None, None, :].expand(1, Q.shape[1], -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(Q[None], K[None], V[None], attn_mask=mask)[0]
+    assert np.max(np.abs(out - ref.permute(1, 0, 2).numpy())) <= 1e-12
+
+
+def _parse_closed_forms():
+    cases, cur = [], None
+    with open(os.path.join(GOLDEN, "attention_closed_form.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            if line.startswith("case "):
+                cur = {"name": line[5:], "k": [], "v": []}
+                cases.append(cur)
+                continue
+            tag, nums = line.split(":", 1)
+            vals = [float(x) for x in nums.split()]
+            if tag in ("k", "v"):
+                cur[tag].append(vals)
+            else:
+                cur[tag] = vals
+    return cases
+
+
+def test_golden_closed_forms():
+    cases = _parse_closed_forms()
+    assert len(cases) >= 3
+    for c in cases:
+        q = np.array(c["q"])[None, None, :]
+        k = np.array(c["k"])[:, None, :]
+        v = np.array(c["v"])[:, None, :]
+        out = orc.attention_rows(q, k, v)[0, 0]
+        assert np.allclose(out, c["out"], rtol=0, atol=1e-14), (c["name"], out)
+
+
+def test_softmax_rows_sum_to_one():
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((7, 3, 16)) * 4
+    k = rng.standard_normal((50, 3, 16))
+    v = rng.standard_normal((50, 3, 16))
+    _, p = orc.attention_rows(q, k, v, return_probs=True)
+    assert np.max(np.abs(p.sum(-1) - 1.0)) <= 1e-12
+    assert np.all(p >= 0)
+
+
+@pytest.mark.parametrize("R", [2, 3, 7])
+def test_r_split_rows_and_heads_bit_identical(R):
+    cfg = _cfg(n_heads=7, head_dim=16, n_video=20, n_audio=3, n_cond=4, history_units=3)
+    cache = orc.UnitCache(cfg)
+    _fill(cache, cfg, [0, 1, 2, 3, 4], seed=2)
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q = _bits(2, synth.KIND_Q, qs, 4)
+    kn = _bits(2, synth.KIND_K_NEW, qs, 4)
+    vn = _bits(2, synth.KIND_V_NEW, qs, 4)
+    st, full = cache.unit_attention(1, 4, q, kn, vn)
+    assert st == orc.OK
+    k, v, _ = cache.visible_kv(1, 4)
+    qf = orc.bf16_to_f64(q)
+    row_parts = np.array_split(np.arange(cfg.n_query), R)
+    by_rows = np.concatenate([orc.attention_rows(qf[rp], k, v) for rp in row_parts], axis=0)
+    assert np.array_equal(by_rows, full)
+    head_parts = np.array_split(np.arange(cfg.n_heads), R)
+    by_heads = np.concatenate([orc.attention_rows(qf[:, hp], k[:, hp], v[:, hp]) for hp in head_parts], axis=1)
+    assert np.array_equal(by_heads, full)
+
+
+def test_zero_query_gives_mean_of_visible_values():
+    """q = 0 makes every logit 0, so out is the plain mean of the visible V rows:
+    this pins the visible key set and its size (the window and the segments)."""
+    cfg = _cfg(history_units=2)
+    cache = orc.UnitCache(cfg)
+    _fill(cache, cfg, [0, 1, 2, 3, 4], skip_latent=(2,))
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q = np.zeros(qs, np.uint16)
+    kn = _bits(1, synth.KIND_K_NEW, qs, 4)
+    vn = _bits(1, synth.KIND_V_NEW, qs, 4)
+    st, out = cache.unit_attention(0, 4, q, kn, vn)
+    assert st == orc.OK
+    # visible: units 2, 3, 4; unit 2 has no committed latent
+    cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+    ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    rows = [orc.bf16_to_f64(_bits(1, synth.KIND_COND_V, cs, u))[0] for u in (2, 3, 4)]
+    rows.append(orc.bf16_to_f64(_bits(1, synth.KIND_COMMIT_V, ls, 3))[0])
+    rows.append(orc.bf16_to_f64(vn))
+    allv = np.concatenate(rows)
+    assert allv.shape[0] == 3 * cfg.n_cond + 2 * cfg.n_query
+    want = allv.mean(axis=0)
+    assert np.max(np.abs(out - want[None])) <= 1e-14
+
+
+def test_constant_values_and_single_key():
+    # all V rows equal c -> out = c
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((5, 2, 8))
+    k = rng.standard_normal((30, 2, 8))
+    v = np.full((30, 2, 8), 0.375)
+    assert np.max(np.abs(orc.attention_rows(q, k, v) - 0.375)) <= 1e-15
+    # the smallest cache: no conditioning, one latent token, no history -> out = v_new
+    cfg = _cfg(n_video=1, n_audio=0, n_cond=0, history_units=0, n_layers=1)
+    cache = orc.UnitCache(cfg)
+    e = np.zeros((1, 0, cfg.n_heads, cfg.head_dim), np.uint16)
+    assert cache.append(0, orc.SEG_COND, e, e) == orc.OK
+    qs = (1, cfg.n_heads, cfg.head_dim)
+    vn = _bits(4, synth.KIND_V_NEW, qs)
+    st, out = cache.unit_attention(0, 0, _bits(4, synth.KIND_Q, qs), _bits(4, synth.KIND_K_NEW, qs), vn)
+    assert st == orc.OK
+    assert np.array_equal(out, orc.bf16_to_f64(vn))
+
+
+def test_masked_units_do_not_leak():
+    """Values far outside the window are huge; a mask error would show up at once."""
+    cfg = _cfg(history_units=1)
+    cache = orc.UnitCache(cfg)
+    cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+    ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    huge = np.full(cs, 0x4780, np.uint16)           # 65536
+    huge_l = np.full(ls, 0x4780, np.uint16)
+    small = np.full(cs, 0x3F80, np.uint16)          # 1
+    small_l = np.full(ls, 0x3F80, np.uint16)
+    assert cache.append(0, orc.SEG_COND, small, huge) == orc.OK
+    assert cache.append(0, orc.SEG_LATENT, small_l, huge_l) == orc.OK
+    for u in (1, 2):
+        assert cache.append(u, orc.SEG_COND, small, small) == orc.OK
+    assert cache.append(1, orc.SEG_LATENT, small_l, small_l) == orc.OK
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    st, out = cache.unit_attention(1, 2, _bits(3, synth.KIND_Q, qs), np.full(qs, 0x3F80, np.uint16),
+                                   np.full(qs, 0x3F80, np.uint16))
+    assert st == orc.OK
+    assert np.max(np.abs(out - 1.0)) <= 1e-15      # every visible value is 1
+
+
+def test_ring_slot_table_closed_form():
+    cfg = _cfg(history_units=3)                      # C = 4
+    cache = orc.UnitCache(cfg)
+    units = [0, 1, 2, 3, 4, 5, 7, 8, 9, 10, 13]
+    _fill(cache, cfg, units, commit=False)
+    C = cfg.slots
+    want = [-1] * C
+    for u in units:
+        want[u % C] = u
+    assert cache.slot_table() == want
+
+
+def test_error_rules():
+    cfg = _cfg(history_units=2)                      # C = 3
+    cache = orc.UnitCache(cfg)
+    qs = (cfg.n_query, cfg.n_heads, cfg.head_dim)
+    z = np.zeros(qs, np.uint16)
+    assert cache.unit_attention(0, 0, z, z, z)[0] == orc.ERR_NOT_READY   # nothing appended
+    _fill(cache, cfg, [0, 1, 2, 3, 4], commit=False)
+    cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+    ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    zc, zl = np.zeros(cs, np.uint16), np.zeros(ls, np.uint16)
+    assert cache.append(3, orc.SEG_COND, zc, zc) == orc.ERR_UNIT_ORDER
+    assert cache.append(4, orc.SEG_COND, zc, zc) == orc.OK               # same unit again
+    assert cache.append(1, orc.SEG_LATENT, zl, zl) == orc.ERR_EVICTED    # slot 1 now holds unit 4
+    assert cache.append(2, orc.SEG_LATENT, zl, zl) == orc.OK
+    assert cache.append(5, orc.SEG_LATENT, zl, zl) == orc.ERR_NOT_READY
+    assert cache.unit_attention(0, 3, z, z, z)[0] == orc.ERR_UNIT_ORDER
+    assert cache.unit_attention(0, 5, z, z, z)[0] == orc.ERR_NOT_READY
+    assert cache.unit_attention(2, 4, z, z, z)[0] == orc.ERR_ARG         # layer out of range
+    assert cache.read(0, 3, orc.SEG_LATENT)[0] == orc.ERR_NOT_READY
+    assert cache.read(0, 0, orc.SEG_COND)[0] == orc.ERR_EVICTED
+    assert cache.read(0, 4, orc.SEG_COND)[0] == orc.OK
+    assert cache.append(-1, orc.SEG_COND, zc, zc) == orc.ERR_ARG
