@@ -1,0 +1,509 @@
+"""Benchmark of the performer unit step on B200.
+
+One step = one full 640x368 unit of the performer: append the thinker's
+conditioning slice, then for each of the 4 flow-matching Euler steps run the 40
+layers' block-causal attention over the 64-unit history (each call first writes
+the current latent tokens' K/V into the cache), then the Euler update of the
+unit latent; finally commit the unit's latent K/V.  Inputs are seeded synthetic
+N(0,1) bf16 tensors resident in HBM before the timed region; the 50.9 GB cache
+and the per-call inputs are far larger than L2, so no flush is needed.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Under torchrun (N > 1) every rank runs an
+independent replica (the unit step has no cross-GPU exchange on one GPU's
+work), the step time is the max over ranks and ``value`` aggregates all ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "block-causal unit-attention TFLOP/s & ms per 640×368 unit on 1 B200 (% of bf16 peak)"
+UNIT = "TFLOP/s"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "unit_attention_traffic.txt")
+KERNEL_SOURCES = ["kv_cache_serving_ws_b200/csrc/attention.cu", "kv_cache_serving_ws_b200/csrc/sm100.cuh",
+                  "kv_cache_serving_ws_b200/csrc/kernels.cuh", "kv_cache_serving_ws_b200/csrc/tmem_ldst.cuh"]
+
+
+# ------------------------------------------------------------ multi-rank --
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity when there is one rank)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device_index=None):
+    if world <= 1:
+        return
+    import torch.distributed as dist
+    if device_index is not None and dist.get_backend() == "nccl":
+        dist.barrier(device_ids=[device_index])
+    else:
+        dist.barrier()
+
+
+def aggregate(per_rank_flops: float, world: int, step_s_max: float, steps: int) -> float:
+    """Whole-job TFLOP/s: every rank's work over the slowest rank's time."""
+    return per_rank_flops * world * steps / step_s_max / 1e12 / steps if step_s_max > 0 else 0.0
+
+
+# ---------------------------------------------------------------- helpers --
+
+def peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return {"hbm": p["hbm_gbs"], "bf16": p["bf16_tflops"], "bf16_sustained": p["bf16_tflops_sustained"],
+                "source": "measured"}
+    except Exception:
+        return {"hbm": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken
+    on the current kernel source; else None."""
+    try:
+        kv = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if "=" in line and not line.startswith("#"):
+                    k, v = line.strip().split("=", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_sha") != kernel_source_sha():
+            return None
+        return float(kv["traffic_bytes_per_full_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = max(smax, float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax or None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our arm --
+
+def run_ours(args, rank, local_rank, world):
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200 import synth
+    from kv_cache_serving_ws_b200.workloads import FULL, GpuSession, key
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = FULL
+    L, S = w.n_layers, w.steps
+    g = GpuSession(w, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # ---- resident inputs: one unit's worth, reused by every timed unit
+    qs = (w.n_query, w.n_heads, w.head_dim)
+    n_lat = w.n_query * w.n_heads * w.head_dim
+    bf = torch.bfloat16
+    q_all = torch.empty((S, L) + qs, dtype=bf, device=dev)
+    kn_all, vn_all = torch.empty_like(q_all), torch.empty_like(q_all)
+    for s in range(S):
+        for l in range(L):
+            g.fill(q_all[s, l], key(w, synth.KIND_Q, w.unit, l, s))
+            g.fill(kn_all[s, l], key(w, synth.KIND_K_NEW, w.unit, l, s))
+            g.fill(vn_all[s, l], key(w, synth.KIND_V_NEW, w.unit, l, s))
+    vel = torch.empty((S, n_lat), dtype=bf, device=dev)
+    for s in range(S):
+        g.fill(vel[s], key(w, synth.KIND_VEL, w.unit, 0, s))
+    x0 = torch.empty(n_lat, dtype=bf, device=dev)
+    g.fill(x0, key(w, synth.KIND_X, w.unit))
+    x = x0.clone()
+    out = torch.empty(qs, dtype=bf, device=dev)
+    cond_k = torch.empty_like(g.cond_k)
+    cond_v = torch.empty_like(g.cond_v)
+    g.fill(cond_k, key(w, synth.KIND_COND_K, w.unit))
+    g.fill(cond_v, key(w, synth.KIND_COND_V, w.unit))
+    commit_k, commit_v = g.commit_buffers()
+
+    # ---- steady-state history: 64 committed units, each with its own data
+    for u in range(0, w.unit):
+        g.append_cond(u)
+        g.commit(u)
+    g.fill(commit_k, key(w, synth.KIND_COMMIT_K, w.unit))
+    g.fill(commit_v, key(w, synth.KIND_COMMIT_V, w.unit))
+    torch.cuda.synchronize()
+
+    h = g.h
+    next_unit = [w.unit]
+
+    def unit_step(x_dev, inputs=None, after_call=None, vel_of=None):
+        """One unit: conditioning append, S x L attention calls with Euler updates, commit."""
+        u = next_unit[0]
+        ws.ws_cache_append(h, u, ws.WS_SEG_COND, cond_k, cond_v)
+        for s in range(S):
+            for l in range(L):
+                q, kn, vn = (q_all[s, l], kn_all[s, l], vn_all[s, l]) if inputs is None else inputs(s, l)
+                ws.ws_unit_attention(h, l, u, q, kn, vn, out)
+                if after_call is not None:
+                    after_call(s, l)
+            ws.ws_flow_step(x_dev, vel[s] if vel_of is None else vel_of(s), w.dt)
+        ws.ws_cache_append(h, u, ws.WS_SEG_LATENT, commit_k, commit_v)
+        next_unit[0] = u + 1
+
+    for _ in range(args.warmup):
+        unit_step(x)
+    assert ws.ws_sync(h, check=False) == ws.WS_OK
+    ws.ws_profile_enable(h, True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, local_rank)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            unit_step(x)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world, local_rank)
+    step_ms = e0.elapsed_time(e1) / args.steps
+    prof = ws.ws_profile_read(h)
+    ws.ws_profile_enable(h, False)
+    st = ws.ws_sync(h, check=False)
+    if st != ws.WS_OK:
+        raise RuntimeError(f"device status after the timed region: {ws.status_string(st)}")
+    step_ms_max = max_over_ranks(step_ms, world, dev)
+    flops_unit = w.flops_per_call() * L * S
+    value = aggregate(flops_unit, world, step_ms_max / 1e3, 1)
+
+    # ---- dominant kernel: attention, event-timed per launch inside the timed region
+    pk = peaks()
+    n_attn = prof["attention_launches"]
+    attn_ms_avg = prof["attention_ms"] / max(1, n_attn)
+    achieved = w.flops_per_call() / (attn_ms_avg / 1e3) / 1e12
+    traffic = recorded_traffic()
+    roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
+                "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": traffic,
+                "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
+    launches_per_step = (2 + L * S * (2 + (1 if prof["last_n_split"] > 1 else 0)) + S)
+
+    # ---- HBM-bound kernels, timed on their own on the same stream
+    extra = hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit)
+
+    # ---- end to end: the same unit step with inputs copied from pinned host memory each step
+    e2e = run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, world, local_rank, flops_unit)
+
+    clocks = clk.summary()
+    g.close()
+    return {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms_max, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "layers": L, "euler_steps": S, "heads": w.n_heads, "head_dim": w.head_dim,
+                   "query_tokens": w.n_query, "video_tokens": w.n_video, "audio_tokens": w.n_audio,
+                   "cond_tokens": w.n_cond, "history_units": w.history_units, "keys_per_query": w.n_keys,
+                   "cache_gb": round(g_cache_bytes(w) / 1e9, 1), "tflop_per_unit": round(flops_unit / 1e12, 2),
+                   "unit_budget_ms": 160, "l2": "no flush: inputs larger than L2 (the 50.9 GB cache is streamed)",
+                   "parallelism": f"replicas x{world}", "attention_splits": prof["last_n_split"],
+                   "attention_ctas": prof["last_ctas"]},
+        "roofline": roofline,
+        "kernels": extra,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+
+
+def g_cache_bytes(w):
+    return w.n_layers * 2 * w.n_heads * (w.history_units + 1) * w.tokens_per_unit * w.head_dim * 2
+
+
+def hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit):
+    """Append (all-layer latent commit) and Euler update timed on their own."""
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    u = next_unit[0] - 1                         # the last committed unit: still resident
+    reps = 10
+    ws.ws_cache_append(g.h, u, ws.WS_SEG_LATENT, commit_k, commit_v)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        ws.ws_cache_append(g.h, u, ws.WS_SEG_LATENT, commit_k, commit_v)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    commit_ms = e0.elapsed_time(e1) / reps
+    commit_bytes = 2 * 2 * commit_k.numel() * 2  # K and V, read + write
+    # Euler on a buffer larger than L2 (2^28 elements = 1.5 GB moved per call)
+    n = 1 << 28
+    xb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    vb = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    g.fill(xb, 12345)
+    g.fill(vb, 54321)
+    ws.ws_flow_step(xb, vb, 0.25)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(reps):
+        ws.ws_flow_step(xb, vb, 0.25)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    euler_ms = e0.elapsed_time(e1) / reps
+    euler_bytes = n * 6
+    del xb, vb
+    hbm = pk["hbm"]
+    return {
+        "latent_commit": {"bytes": commit_bytes, "ms": round(commit_ms, 4),
+                          "GB/s": round(commit_bytes / commit_ms / 1e6, 1),
+                          "frac_of_measured_hbm": round(commit_bytes / commit_ms / 1e6 / hbm, 4),
+                          "frac_of_8TBs": round(commit_bytes / commit_ms / 1e6 / 8000, 4)},
+        "euler_2^28": {"bytes": euler_bytes, "ms": round(euler_ms, 4), "GB/s": round(euler_bytes / euler_ms / 1e6, 1),
+                       "frac_of_measured_hbm": round(euler_bytes / euler_ms / 1e6 / hbm, 4),
+                       "frac_of_8TBs": round(euler_bytes / euler_ms / 1e6 / 8000, 4)},
+    }
+
+
+def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, world, local_rank, flops_unit):
+    """Same unit step, each step's inputs copied host->device from pinned memory on a
+    copy stream (double-buffered per layer-step) and the final latent copied back."""
+    L, S = w.n_layers, w.steps
+    n_sets = 8                                   # distinct host input sets, cycled
+    qs = q_all.shape[2:]
+    host = torch.empty((n_sets, 3) + tuple(qs), dtype=torch.bfloat16, pin_memory=True)
+    for i in range(n_sets):
+        s, l = divmod(i, L)
+        host[i, 0].copy_(q_all[s, l])
+        host[i, 1].copy_(kn_all[s, l])
+        host[i, 2].copy_(vn_all[s, l])
+    host_vel = vel.cpu().pin_memory()
+    host_x = x0.cpu().pin_memory()
+    host_x_out = torch.empty_like(host_x).pin_memory()
+    dbuf = torch.empty((2, 3) + tuple(qs), dtype=torch.bfloat16, device=dev)
+    dvel = torch.empty_like(vel)
+    x = torch.empty_like(x0)
+    comp = torch.cuda.current_stream()
+    copy = torch.cuda.Stream(device=dev)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
+    order = [(s, l) for s in range(S) for l in range(L)]
+
+    def one_unit():
+        with torch.cuda.stream(copy):
+            x.copy_(host_x, non_blocking=True)
+            dvel.copy_(host_vel, non_blocking=True)
+            first = torch.cuda.Event()
+            first.record(copy)
+
+        def stage(i):
+            s, l = order[i]
+            b = i % 2
+            with torch.cuda.stream(copy):
+                if i >= 2:
+                    copy.wait_event(free[b])
+                dbuf[b].copy_(host[(s * L + l) % n_sets], non_blocking=True)
+                ready[b].record(copy)
+
+        stage(0)
+        comp.wait_event(first)
+        pos = {sl: i for i, sl in enumerate(order)}
+
+        def inputs(s, l):
+            i = pos[(s, l)]
+            if i + 1 < len(order):
+                stage(i + 1)
+            comp.wait_event(ready[i % 2])
+            return dbuf[i % 2, 0], dbuf[i % 2, 1], dbuf[i % 2, 2]
+
+        def after_call(s, l):
+            free[pos[(s, l)] % 2].record(comp)
+
+        unit_step(x, inputs, after_call, lambda s: dvel[s])
+        host_x_out.copy_(x, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        one_unit()
+    torch.cuda.synchronize()
+    barrier(world, local_rank)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(comp)
+    for _ in range(args.steps):
+        one_unit()
+    e1.record(comp)
+    torch.cuda.synchronize()
+    barrier(world, local_rank)
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
+    h2d = (L * S * 3 * q_all[0, 0].numel() + vel.numel() + x0.numel()) * 2
+    d2h = x0.numel() * 2
+    return {"value": round(aggregate(flops_unit, world, ms / 1e3, 1), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "note": "conditioning and commit K/V stay device-resident; q, k_new, v_new, velocities and x cross PCIe"}
+
+
+# ------------------------------------------------------- the oracle arm --
+
+def oracle_sample(target_s: float, max_rows=None):
+    """Time the fp64 oracle on a bounded sample of the same workload: one head of one
+    layer-step, as many query rows as fit in about target_s seconds."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    import numpy as np
+
+    from kv_cache_serving_ws_b200.workloads import FULL
+    from oracle_side import oracle_cache
+    w = FULL
+    cache, q, kn, vn = oracle_cache(w, 17, [0], 1)
+    # probe a few rows, then size the sample
+    t0 = time.perf_counter()
+    st, _ = cache.unit_attention(0, w.unit, q, kn, vn, rows=[0, 1])
+    t_row = (time.perf_counter() - t0) / 2
+    rows = max(2, min(w.n_query, int(target_s / max(t_row, 1e-6))))
+    if max_rows:
+        rows = min(rows, max_rows)
+    t0 = time.perf_counter()
+    st, _ = cache.unit_attention(0, w.unit, q, kn, vn, rows=list(range(rows)))
+    dt = time.perf_counter() - t0
+    assert st == 0
+    flops = 4.0 * rows * w.n_keys * 1 * w.head_dim
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"1 head x {rows} query rows of one layer-step of {w.name} ({w.n_keys} keys), "
+                      f"{dt:.1f} s; ms per unit extrapolated x{w.n_heads} heads x{w.n_query/rows:.2f} rows "
+                      f"x{w.n_layers * w.steps} layer-steps = {dt * w.n_heads * (w.n_query / rows) * w.n_layers * w.steps * 1e3:.0f} ms",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return None
+    samples = []
+    for _ in range(args.warmup):
+        oracle_sample(1.0, max_rows=4)
+    t_all = 0.0
+    for _ in range(args.steps):
+        s = oracle_sample(args.ref_step_seconds)
+        samples.append(s)
+        t_all += s["seconds"]
+    val = statistics.median([s["value"] for s in samples])
+    base = dict(samples[-1])
+    base["value"] = val
+    from kv_cache_serving_ws_b200.workloads import FULL
+    return {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(t_all / args.steps * 1e3, 1), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": FULL.name, "sample": base["sample"]},
+            "cpu_baseline": base,
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    rank, local_rank, world = dist_env()
+    if args.impl == "reference":
+        line = run_reference(args)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, local_rank, world)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = oracle_sample(args.cpu_baseline_seconds)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,234 @@
+/*
+ * ws.h -- C ABI of the performer unit-step library (libws.so).
+ *
+ * The library implements, on one B200 (sm_100a), the per-unit denoising step of
+ * the Wan-Streamer v0.2 performer as described on the pages about that report:
+ *
+ *   - a preallocated K/V history cache into which each incoming thinker K/V
+ *     slice is written in place ("Wan-Streamer v0.2：更高分辨率，相同延迟",
+ *     paper.rainbus.top, section 前置知识, entry K/V缓存预分片; "Technical
+ *     Summary: Wan-Streamer v0.2", gist.science, section Methodology, item 2,
+ *     K/V Handling), and into which the generated latents are committed after
+ *     each unit (paper.rainbus.top, section 核心方法);
+ *   - block-causal attention at the granularity of one 160 ms streaming unit:
+ *     a token sees all tokens of its own unit and of earlier units, none of a
+ *     later one ("通义实验室发布 Wan-Streamer v0.2…", remio.ai, section
+ *     为什么端到端模型对级联式 AI 智能体构成挑战), using cached K/V instead of
+ *     recomputing the history (remio.ai, section 思考者与执行者的分工掩盖了更高分辨率的成本);
+ *   - the flow-matching Euler update of the latent, x <- x + dt*v
+ *     (paper.rainbus.top, section 核心方法, flow-matching latent generation).
+ *
+ * Everything runs on one GPU with no sharding; the pages split the performer
+ * across GPUs with Ulysses context parallelism, which this library does not do.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - bf16 tensors are passed as pointers to their 16-bit patterns (uint16_t).
+ *  - Every tensor pointer is DEVICE memory owned by the caller, 16-byte aligned
+ *    (else WS_ERR_ALIGN), dense row-major in the layout stated at each call.
+ *  - Calls are asynchronous and ordered on the given stream (NULL = the legacy
+ *    default stream).  None synchronises, except ws_sync and ws_cache_destroy.
+ *    The caller keeps inputs alive and unmodified until the work on the stream
+ *    has consumed them.
+ *  - Argument errors are detected on the host before any launch and leave all
+ *    state unchanged.  A CUDA launch error returns WS_ERR_CUDA.  Errors found by
+ *    a kernel (a bounded wait that ran out) are stored in the cache's device
+ *    status word and reported by the next ws_sync.
+ *  - The library owns the cache memory, its slot table, the split-K workspace and
+ *    the status word.  A cache belongs to the device that was current when it was
+ *    created; calls on it must be made with that device current.
+ *
+ * Shapes: L = n_layers, H = n_heads, D = head_dim (64 or 128),
+ * Nq = n_video + n_audio (latent tokens generated per unit), Nc = n_cond
+ * (thinker conditioning tokens per unit), T = Nc + Nq (tokens per unit slot),
+ * U = history_units, C = U + 1 (ring slots).
+ */
+#ifndef WS_H
+#define WS_H
+
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned by every call. */
+enum {
+  WS_OK = 0,
+  WS_ERR_ARG = -1,             /* bad pointer, size, layer, segment or configuration */
+  WS_ERR_ALIGN = -2,           /* a tensor pointer is not 16-byte aligned */
+  WS_ERR_OOM = -3,             /* device allocation failed in ws_cache_create */
+  WS_ERR_UNIT_ORDER = -4,      /* unit older than the newest conditioned unit */
+  WS_ERR_EVICTED = -5,         /* the unit's slot has been reused by a newer unit */
+  WS_ERR_NOT_READY = -6,       /* the unit (or its latent segment) was never written */
+  WS_ERR_CUDA = -7,            /* a CUDA runtime call or launch failed */
+  WS_ERR_DEVICE_TIMEOUT = -8,  /* a kernel's bounded wait ran out (reported by ws_sync) */
+  WS_ERR_UNSUPPORTED = -9      /* valid request outside what this build supports (e.g. D not 64/128) */
+};
+
+/* Segments of a unit slot: the thinker's conditioning tokens, then the unit's latent tokens. */
+enum { WS_SEG_COND = 0, WS_SEG_LATENT = 1 };
+
+typedef struct ws_cache ws_cache_t;   /* opaque, library-owned */
+
+typedef struct {
+  int32_t n_layers;       /* L >= 1 */
+  int32_t n_heads;        /* H >= 1 */
+  int32_t head_dim;       /* D: 64 or 128 */
+  int32_t n_video;        /* latent video tokens per unit (>= 0) */
+  int32_t n_audio;        /* latent audio tokens per unit (>= 0), unsharded, same attention set */
+  int32_t n_cond;         /* thinker K/V conditioning tokens per unit (>= 0) */
+  int32_t history_units;  /* U >= 0: earlier units a query can see; the ring holds C = U + 1 */
+} ws_cache_config;
+
+/*
+ * ws_cache_create -- allocate and zero a K/V history cache on the current device.
+ *
+ * Memory: K and V planes [L][2][H][C*T][D] bf16 (plane (l, 0, h) holds K of
+ * layer l, head h; (l, 1, h) holds V), token rows of slot s at [s*T, (s+1)*T):
+ * first the Nc conditioning rows, then the Nq latent rows (video, then audio).
+ * Also a split-K workspace and a device status word.  Nq must be >= 1; the
+ * total row count C*T must fit in 2^31.  On success *out receives the handle.
+ * Errors: WS_ERR_ARG (NULL pointer, bad sizes), WS_ERR_UNSUPPORTED (D),
+ * WS_ERR_OOM, WS_ERR_CUDA.  The zero fill is ordered on `stream`.
+ */
+int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t stream);
+
+/* Synchronise the device, free everything the handle owns, free the handle. NULL is a no-op. */
+int ws_cache_destroy(ws_cache_t* h);
+
+/*
+ * ws_cache_append -- write one incoming K/V slice in place.
+ *
+ * seg == WS_SEG_COND: the thinker's conditioning slice of `unit`,
+ *   k_slice, v_slice: [L][Nc][H][D].  Units are non-decreasing: unit < newest
+ *   returns WS_ERR_UNIT_ORDER.  unit > newest starts a new unit: it claims slot
+ *   unit mod C (evicting the unit that held it) and becomes the newest.
+ *   unit == newest rewrites its conditioning rows.
+ * seg == WS_SEG_LATENT: the commit of `unit`'s generated latents, all layers,
+ *   k_slice, v_slice: [L][Nq][H][D] (committed history, paper.rainbus.top,
+ *   section 核心方法).  The unit must be resident: WS_ERR_EVICTED if its slot
+ *   holds a newer unit, WS_ERR_NOT_READY if its conditioning slice was never
+ *   appended.
+ * The copy is a bit-exact bf16 copy.  Errors: WS_ERR_ARG, WS_ERR_ALIGN, the
+ * unit errors above, WS_ERR_CUDA.
+ */
+int ws_cache_append(ws_cache_t* h, int64_t unit, int seg,
+                    const uint16_t* k_slice, const uint16_t* v_slice, cudaStream_t stream);
+
+/*
+ * ws_unit_attention -- one layer of block-causal attention for the newest unit.
+ *
+ * First writes k_new, v_new ([Nq][H][D], the current, still-noisy latent
+ * tokens' K/V of this layer) into the unit's latent rows of `layer`; then, for
+ * every head h and query row i of q ([Nq][H][D]),
+ *     out[i][h] = sum_j softmax_j(q[i][h] . k_j[h] / sqrt(D)) v_j[h]
+ * over the visible keys j: for every resident unit u' with
+ * unit - U <= u' <= unit, its Nc conditioning rows, and its Nq latent rows of
+ * this layer if they have been written (by this call for u' = unit, by an
+ * earlier commit or attention call otherwise).  Within a unit the attention is
+ * bidirectional (video and audio together); across units it is causal.
+ * out: [Nq][H][D] bf16 (written, not accumulated).  Arithmetic: bf16 tensor-core
+ * products with fp32 accumulation, fp32 online softmax, P rounded to bf16
+ * before the P.V product, RNE to bf16 at the end.
+ * Errors: WS_ERR_ARG (layer, pointers), WS_ERR_ALIGN, WS_ERR_NOT_READY (unit is
+ * newer than the newest conditioned unit), WS_ERR_UNIT_ORDER (unit is older
+ * than the newest: the stream has moved on), WS_ERR_CUDA.
+ */
+int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit,
+                      const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                      uint16_t* out, cudaStream_t stream);
+
+/*
+ * ws_flow_step -- fused flow-matching Euler update, in place:
+ *     x[i] <- RN_bf16( fl64( x[i] + fl64(dt * v[i]) ) ),   0 <= i < n
+ * (paper.rainbus.top, section 核心方法).  dt*v is exact in fp64; the sum is
+ * rounded once to fp64 and once to bf16, round-to-nearest-even; every NaN
+ * result is stored as 0x7FC0.  x and v: n bf16 elements, 16-byte aligned,
+ * x and v must not overlap unless x == v.  n == 0 is a no-op.
+ * Errors: WS_ERR_ARG (NULL with n > 0, n < 0), WS_ERR_ALIGN, WS_ERR_CUDA.
+ */
+int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream);
+
+/*
+ * ws_cache_read -- copy one segment of one resident unit and layer out of the
+ * cache (a bit-exact readback for tests and checkpoints).  k_out, v_out:
+ * [Nc][H][D] for WS_SEG_COND, [Nq][H][D] for WS_SEG_LATENT.
+ * Errors: WS_ERR_ARG, WS_ERR_ALIGN, WS_ERR_EVICTED, WS_ERR_NOT_READY (never
+ * appended, or the latent rows of that layer were never written), WS_ERR_CUDA.
+ */
+int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg,
+                  uint16_t* k_out, uint16_t* v_out, cudaStream_t stream);
+
+/* Copy the slot table (C entries: the unit held by each slot, -1 = empty) to host memory. */
+int ws_cache_slot_table(const ws_cache_t* h, int64_t* slot_unit_host);
+
+/* Sizes derived from the configuration. */
+typedef struct {
+  int32_t slots;               /* C */
+  int32_t tokens_per_unit;     /* T */
+  int32_t n_query;             /* Nq */
+  int64_t newest_unit;         /* -1 before the first append */
+  uint64_t cache_bytes;        /* K and V planes */
+  uint64_t workspace_bytes;    /* split-K partials */
+} ws_cache_info;
+
+int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info);
+
+/*
+ * ws_cache_set_splits -- number of key-range splits of each attention call
+ * (split-K partials merged by a second kernel).  0 = automatic (chosen to fill
+ * the 148 SMs), 1..16 forces that count (clamped to the number of key tiles).
+ */
+int ws_cache_set_splits(ws_cache_t* h, int n_split);
+
+/*
+ * ws_sync -- synchronise `stream`, then read and clear the device status word.
+ * Returns WS_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the
+ * last ws_sync, WS_ERR_CUDA on a CUDA error, else WS_OK.
+ */
+int ws_sync(ws_cache_t* h, cudaStream_t stream);
+
+/* Static, human-readable text of a status code. */
+const char* ws_status_string(int status);
+
+/*
+ * Launch accounting of the attention path, for benchmarks.  While enabled, the
+ * library records a CUDA event pair around each attention kernel and each
+ * combine kernel it launches (on the caller's stream).  ws_profile_read
+ * synchronises those events and returns the totals since the last reset.
+ */
+typedef struct {
+  int64_t attention_launches;
+  double attention_ms;         /* sum of event-timed durations */
+  int64_t combine_launches;
+  double combine_ms;
+  int64_t latent_write_launches;
+  double latent_write_ms;
+  int32_t last_n_split;        /* split count of the last attention call */
+  int32_t last_ctas;           /* CTAs of the last attention launch */
+  int64_t last_keys;           /* visible keys of the last attention call */
+} ws_profile;
+
+int ws_profile_enable(ws_cache_t* h, int enable);   /* enabling resets the totals */
+int ws_profile_read(ws_cache_t* h, ws_profile* out);
+
+/*
+ * ws_plan_visible -- host-only planning step of ws_unit_attention, exposed for
+ * tests: the key rows of one (layer, head) plane that a query of `unit` sees,
+ * as maximal runs of consecutive rows [row_begin[i], row_begin[i] + rows[i]).
+ * slot_unit: C entries as from ws_cache_slot_table; latent_ready: C*L bytes,
+ * entry [s*L + l] nonzero when slot s holds latent rows of layer l (the query
+ * unit's own latent rows count as written).  Touches no GPU.
+ * Errors: WS_ERR_ARG; WS_ERR_UNSUPPORTED if more than max_runs runs are needed.
+ */
+int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit,
+                    const uint8_t* latent_ready, int layer, int64_t unit,
+                    int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WS_H */

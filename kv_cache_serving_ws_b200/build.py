@@ -1,0 +1,73 @@
+"""Build the CUDA libraries in-tree for sm_100a with nvcc.
+
+    python -m kv_cache_serving_ws_b200.build [--force] [--ptxas-info]
+
+produces, next to this file:
+  libws.so        the unit-step library (include/ws.h)
+  libws_synth.so  the device input generator (include/ws_synth.h)
+"""
+from __future__ import annotations
+
+import argparse
+import os
+import shutil
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+INCLUDE = os.path.join(ROOT, "include")
+
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "-cudart", "static",
+         "--expt-relaxed-constexpr", "-I", INCLUDE]
+
+LIBS = {
+    "libws.so": ["ws_api.cu", "attention.cu", "copy_kernels.cu", "euler.cu"],
+    "libws_synth.so": ["synth.cu"],
+}
+HEADERS = ["kernels.cuh", "sm100.cuh", "tmem_ldst.cuh"]
+
+
+def nvcc() -> str:
+    for cand in (shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    raise RuntimeError("nvcc not found: the CUDA toolkit is required to build libws")
+
+
+def _stale(out: str, deps: list[str]) -> bool:
+    if not os.path.exists(out):
+        return True
+    t = os.path.getmtime(out)
+    return any(os.path.getmtime(d) > t for d in deps)
+
+
+def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) -> list[str]:
+    built = []
+    hdrs = [os.path.join(CSRC, h) for h in HEADERS] + [os.path.join(INCLUDE, h) for h in ("ws.h", "ws_synth.h")]
+    for lib, srcs in LIBS.items():
+        out = os.path.join(HERE, lib)
+        src_paths = [os.path.join(CSRC, s) for s in srcs]
+        if not force and not ptxas_info and not _stale(out, src_paths + hdrs + [__file__]):
+            continue
+        cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_info else []) + src_paths + ["-o", out]
+        if verbose:
+            print(" ".join(cmd), file=sys.stderr)
+        res = subprocess.run(cmd, capture_output=True, text=True)
+        if res.returncode != 0:
+            raise RuntimeError(f"nvcc failed for {lib}:\n{res.stdout}\n{res.stderr}")
+        if ptxas_info:
+            print(res.stderr, file=sys.stderr)
+        built.append(out)
+    return built
+
+
+if __name__ == "__main__":
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--force", action="store_true")
+    ap.add_argument("--ptxas-info", action="store_true")
+    a = ap.parse_args()
+    for p in build(force=a.force, ptxas_info=a.ptxas_info, verbose=True):
+        print("built", p)

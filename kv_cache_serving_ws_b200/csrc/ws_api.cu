@@ -1,0 +1,477 @@
+// C ABI of libws: handle, argument validation, the unit-slot ring bookkeeping,
+// the visible-row planner and the launches.  Declarations and the contract of
+// every entry point are in include/ws.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <new>
+#include <vector>
+
+#include "../../include/ws.h"
+#include "kernels.cuh"
+
+using namespace ws;
+
+struct EventPool {
+  std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 end
+  int used = 0;
+  int64_t launches = 0;
+  double ms = 0.0;
+  void create(int pairs) {
+    ev.resize(2 * pairs);
+    for (auto& e : ev) cudaEventCreate(&e);
+    used = 0;
+  }
+  void destroy() {
+    for (auto& e : ev) cudaEventDestroy(e);
+    ev.clear();
+  }
+  void flush() {
+    for (int i = 0; i < used; ++i) {
+      cudaEventSynchronize(ev[2 * i + 1]);
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, ev[2 * i], ev[2 * i + 1]) == cudaSuccess) ms += t;
+    }
+    launches += used;
+    used = 0;
+  }
+  cudaEvent_t* next() {
+    if (ev.empty()) return nullptr;
+    if (2 * used >= (int)ev.size()) flush();
+    return &ev[2 * (used++)];
+  }
+};
+
+struct ws_cache {
+  ws_cache_config cfg{};
+  int device = 0;
+  int C = 0, T = 0, Nq = 0;
+  int64_t newest = -1;
+  std::vector<int64_t> slot_unit;     // C
+  std::vector<uint8_t> latent_ready;  // C * L
+  uint16_t* kv = nullptr;
+  size_t kv_bytes = 0;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  size_t ws_bytes = 0;
+  int* d_status = nullptr;
+  CUtensorMap kv_map;
+  int force_splits = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int debug_skip_v_tile = -1;
+  bool profiling = false;
+  EventPool ev_attn, ev_comb, ev_lat;
+  int last_split = 0, last_ctas = 0;
+  int64_t last_keys = 0;
+};
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool config_ok(const ws_cache_config* c) {
+  if (!c) return false;
+  if (c->n_layers < 1 || c->n_heads < 1 || c->head_dim < 1) return false;
+  if (c->n_video < 0 || c->n_audio < 0 || c->n_cond < 0 || c->history_units < 0) return false;
+  const int64_t nq = (int64_t)c->n_video + c->n_audio;
+  if (nq < 1) return false;
+  const int64_t T = nq + c->n_cond;
+  const int64_t C = (int64_t)c->history_units + 1;
+  if (T * C >= (int64_t)1 << 31) return false;
+  if ((int64_t)c->n_layers * 2 * c->n_heads >= (int64_t)1 << 31) return false;
+  if (nq * c->n_heads * (int64_t)c->head_dim >= (int64_t)1 << 40) return false;
+  return true;
+}
+
+// status of `unit` in the ring: resident, evicted (its slot holds a newer unit) or never appended
+int resident(const ws_cache* h, int64_t unit) {
+  if (unit < 0) return WS_ERR_ARG;
+  const int64_t holder = h->slot_unit[(size_t)(unit % h->C)];
+  if (holder == unit) return WS_OK;
+  return holder > unit ? WS_ERR_EVICTED : WS_ERR_NOT_READY;
+}
+
+int plan_runs(const ws_cache_config& cfg, const int64_t* slot_unit, const uint8_t* latent_ready, int layer,
+              int64_t unit, int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs) {
+  const int C = cfg.history_units + 1;
+  const int Nq = cfg.n_video + cfg.n_audio;
+  const int T = cfg.n_cond + Nq;
+  const int64_t lo = unit - cfg.history_units;
+  int n = 0;
+  int64_t run_end = -1;
+  for (int s = 0; s < C; ++s) {
+    const int64_t u = slot_unit[s];
+    if (u < 0 || u < lo || u > unit) continue;
+    const bool lat = (u == unit) || latent_ready[(size_t)s * cfg.n_layers + layer];
+    const int64_t b = (int64_t)s * T;
+    const int64_t e = b + cfg.n_cond + (lat ? Nq : 0);
+    if (e == b) continue;
+    if (n > 0 && b == run_end) {
+      rows[n - 1] += (int32_t)(e - b);
+    } else {
+      if (n == max_runs) return WS_ERR_UNSUPPORTED;
+      row_begin[n] = (int32_t)b;
+      rows[n] = (int32_t)(e - b);
+      ++n;
+    }
+    run_end = e;
+  }
+  *n_runs = n;
+  return WS_OK;
+}
+
+// Number of key-range splits: minimise (waves of CTAs) x (tiles per CTA + fixed
+// per-CTA cost) + the merge pass, over 1..kMaxSplits.
+int choose_splits(int base_ctas, int total_tiles, int head_dim, int forced) {
+  const int cap = std::min(kMaxSplits, std::max(1, total_tiles));
+  if (forced > 0) return std::min(forced, cap);
+  const int sms = sm_count();
+  const double kFixedTiles = 3.0;                       // prologue + epilogue of one CTA, in tile times
+  const double tile_s = 0.8e-6, hbm = 6.5e12;          // rough tile time and HBM rate
+  int best = 1;
+  double best_cost = 1e300;
+  for (int n = 1; n <= cap; ++n) {
+    const int tps = (total_tiles + n - 1) / n;
+    const int n_eff = (total_tiles + tps - 1) / tps;
+    if (n_eff != n) continue;
+    const double waves = std::ceil((double)base_ctas * n / sms);
+    double cost = waves * (tps + kFixedTiles);
+    if (n > 1) cost += 5.0 + (double)n * base_ctas * kBlockM * head_dim * 4.0 / hbm / tile_s;
+    if (cost < best_cost - 1e-9) {
+      best_cost = cost;
+      best = n;
+    }
+  }
+  return best;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? WS_OK : WS_ERR_CUDA; }
+
+void free_all(ws_cache* h) {
+  if (h->kv) cudaFree(h->kv);
+  if (h->part_o) cudaFree(h->part_o);
+  if (h->part_ml) cudaFree(h->part_ml);
+  if (h->d_status) cudaFree(h->d_status);
+  h->ev_attn.destroy();
+  h->ev_comb.destroy();
+  h->ev_lat.destroy();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* ws_status_string(int status) {
+  switch (status) {
+    case WS_OK: return "ok";
+    case WS_ERR_ARG: return "invalid argument";
+    case WS_ERR_ALIGN: return "tensor pointer not 16-byte aligned";
+    case WS_ERR_OOM: return "device allocation failed";
+    case WS_ERR_UNIT_ORDER: return "unit older than the newest conditioned unit";
+    case WS_ERR_EVICTED: return "unit evicted from the ring (its slot holds a newer unit)";
+    case WS_ERR_NOT_READY: return "unit or segment not written yet";
+    case WS_ERR_CUDA: return "CUDA error";
+    case WS_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
+    case WS_ERR_UNSUPPORTED: return "request outside what this build supports";
+    default: return "unknown status";
+  }
+}
+
+int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit, const uint8_t* latent_ready, int layer,
+                    int64_t unit, int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs) {
+  if (!config_ok(cfg) || !slot_unit || !latent_ready || !row_begin || !rows || !n_runs || max_runs < 0)
+    return WS_ERR_ARG;
+  if (layer < 0 || layer >= cfg->n_layers || unit < 0) return WS_ERR_ARG;
+  return plan_runs(*cfg, slot_unit, latent_ready, layer, unit, row_begin, rows, max_runs, n_runs);
+}
+
+int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t stream) {
+  if (!out || !config_ok(cfg)) return WS_ERR_ARG;
+  if (cfg->head_dim != 64 && cfg->head_dim != 128) return WS_ERR_UNSUPPORTED;
+  ws_cache* h = new (std::nothrow) ws_cache();
+  if (!h) return WS_ERR_OOM;
+  h->cfg = *cfg;
+  cudaGetDevice(&h->device);
+  h->Nq = cfg->n_video + cfg->n_audio;
+  h->T = cfg->n_cond + h->Nq;
+  h->C = cfg->history_units + 1;
+  h->slot_unit.assign(h->C, -1);
+  h->latent_ready.assign((size_t)h->C * cfg->n_layers, 0);
+  if (const char* t = std::getenv("WS_WAIT_TIMEOUT_MS")) {
+    const long long ms = std::atoll(t);
+    if (ms > 0) h->timeout_ns = (uint64_t)ms * 1000000ull;
+  }
+  const int L = cfg->n_layers, H = cfg->n_heads, D = cfg->head_dim;
+  const int64_t rows = (int64_t)h->C * h->T;
+  h->kv_bytes = (size_t)L * 2 * H * rows * D * 2;
+  const int64_t rows_pad = (int64_t)((h->Nq + kBlockM - 1) / kBlockM) * kBlockM;
+  const size_t part_o_bytes = (size_t)kMaxSplits * H * rows_pad * D * 4;
+  const size_t part_ml_bytes = (size_t)kMaxSplits * H * rows_pad * 2 * 4;
+  h->ws_bytes = part_o_bytes + part_ml_bytes;
+  int st = WS_OK;
+  if (cudaMalloc(&h->kv, h->kv_bytes) != cudaSuccess || cudaMalloc(&h->part_o, part_o_bytes) != cudaSuccess ||
+      cudaMalloc(&h->part_ml, part_ml_bytes) != cudaSuccess || cudaMalloc(&h->d_status, sizeof(int)) != cudaSuccess)
+    st = WS_ERR_OOM;
+  if (st == WS_OK && (cudaMemsetAsync(h->kv, 0, h->kv_bytes, stream) != cudaSuccess ||
+                      cudaMemsetAsync(h->d_status, 0, sizeof(int), stream) != cudaSuccess))
+    st = WS_ERR_CUDA;
+  if (st == WS_OK && encode_kv_map(&h->kv_map, h->kv, D, rows, (int64_t)L * 2 * H) != 0) st = WS_ERR_CUDA;
+  if (st != WS_OK) {
+    cudaGetLastError();
+    free_all(h);
+    delete h;
+    return st;
+  }
+  *out = h;
+  return WS_OK;
+}
+
+int ws_cache_destroy(ws_cache_t* h) {
+  if (!h) return WS_OK;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  cudaSetDevice(h->device);
+  const cudaError_t e = cudaDeviceSynchronize();
+  free_all(h);
+  delete h;
+  cudaSetDevice(dev);
+  return cuda_status(e);
+}
+
+int ws_cache_append(ws_cache_t* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
+                    cudaStream_t stream) {
+  if (!h || unit < 0 || (seg != WS_SEG_COND && seg != WS_SEG_LATENT)) return WS_ERR_ARG;
+  const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
+  if (n > 0) {
+    if (!k_slice || !v_slice) return WS_ERR_ARG;
+    if (!aligned16(k_slice) || !aligned16(v_slice)) return WS_ERR_ALIGN;
+  }
+  const size_t slot = (size_t)(unit % h->C);
+  if (seg == WS_SEG_COND) {
+    if (unit < h->newest) return WS_ERR_UNIT_ORDER;
+  } else {
+    const int st = resident(h, unit);
+    if (st != WS_OK) return st;
+  }
+  AppendParams p{};
+  p.src_k = k_slice;
+  p.src_v = v_slice;
+  p.cache = h->kv;
+  p.n_layers = h->cfg.n_layers;
+  p.layer0 = 0;
+  p.n_tokens = n;
+  p.n_heads = h->cfg.n_heads;
+  p.head_dim = h->cfg.head_dim;
+  p.plane_rows = (int64_t)h->C * h->T;
+  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  const cudaError_t e = launch_append(p, stream);
+  if (e != cudaSuccess) return WS_ERR_CUDA;
+  if (seg == WS_SEG_COND) {
+    if (unit > h->newest) {
+      h->slot_unit[slot] = unit;
+      std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
+                h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 0);
+      h->newest = unit;
+    }
+  } else {
+    std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
+              h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 1);
+  }
+  return WS_OK;
+}
+
+int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q, const uint16_t* k_new,
+                      const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || unit < 0) return WS_ERR_ARG;
+  if (!q || !k_new || !v_new || !out) return WS_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return WS_ERR_ALIGN;
+  if (h->newest < 0 || unit > h->newest) return WS_ERR_NOT_READY;
+  if (unit < h->newest) return WS_ERR_UNIT_ORDER;
+  const int H = h->cfg.n_heads, D = h->cfg.head_dim, L = h->cfg.n_layers;
+  const size_t slot = (size_t)(unit % h->C);
+
+  // plan first (pure host work), so that an unsupported layout changes nothing
+  std::vector<uint8_t> ready(h->latent_ready);
+  ready[slot * L + layer] = 1;
+  AttnParams p{};
+  int32_t n_runs = 0;
+  int st = plan_runs(h->cfg, h->slot_unit.data(), ready.data(), layer, unit, p.runs.row_begin, p.runs.rows,
+                     kMaxRuns, &n_runs);
+  if (st != WS_OK) return st;
+  p.runs.n_runs = n_runs;
+  int tiles = 0;
+  int64_t keys = 0;
+  for (int r = 0; r < n_runs; ++r) {
+    p.runs.tile_begin[r] = tiles;
+    tiles += (p.runs.rows[r] + kBlockN - 1) / kBlockN;
+    keys += p.runs.rows[r];
+  }
+  p.runs.tile_begin[n_runs] = tiles;
+  p.runs.total_tiles = tiles;
+
+  CUtensorMap q_map;
+  if (encode_q_map(&q_map, q, D, H, h->Nq) != 0) return WS_ERR_CUDA;
+
+  // 1. the current unit's latent K/V of this layer into its slot
+  AppendParams a{};
+  a.src_k = k_new;
+  a.src_v = v_new;
+  a.cache = h->kv;
+  a.n_layers = 1;
+  a.layer0 = layer;
+  a.n_tokens = h->Nq;
+  a.n_heads = H;
+  a.head_dim = D;
+  a.plane_rows = (int64_t)h->C * h->T;
+  a.row0 = (int64_t)slot * h->T + h->cfg.n_cond;
+  cudaEvent_t* ev = h->profiling ? h->ev_lat.next() : nullptr;
+  if (ev) cudaEventRecord(ev[0], stream);
+  if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (ev) cudaEventRecord(ev[1], stream);
+  h->latent_ready[slot * L + layer] = 1;
+
+  // 2. attention (+ merge of split partials)
+  p.n_query = h->Nq;
+  p.n_heads = H;
+  p.n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
+  p.n_split = choose_splits(p.n_qtiles * H, tiles, D, h->force_splits);
+  p.tiles_per_split = (tiles + p.n_split - 1) / p.n_split;
+  p.n_split = (tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  p.plane_k = (layer * 2 + 0) * H;
+  p.plane_v = (layer * 2 + 1) * H;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.out = out;
+  p.part_o = h->part_o;
+  p.part_ml = h->part_ml;
+  p.status = h->d_status;
+  p.timeout_ns = h->timeout_ns;
+  p.debug_skip_v_tile = h->debug_skip_v_tile;
+  ev = h->profiling ? h->ev_attn.next() : nullptr;
+  if (ev) cudaEventRecord(ev[0], stream);
+  int ctas = 0;
+  if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (ev) cudaEventRecord(ev[1], stream);
+  if (p.n_split > 1) {
+    ev = h->profiling ? h->ev_comb.next() : nullptr;
+    if (ev) cudaEventRecord(ev[0], stream);
+    if (launch_combine(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
+    if (ev) cudaEventRecord(ev[1], stream);
+  }
+  h->last_split = p.n_split;
+  h->last_ctas = ctas;
+  h->last_keys = keys;
+  return WS_OK;
+}
+
+int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {
+  if (n < 0) return WS_ERR_ARG;
+  if (n == 0) return WS_OK;
+  if (!x || !v) return WS_ERR_ARG;
+  if (!aligned16(x) || !aligned16(v)) return WS_ERR_ALIGN;
+  return cuda_status(launch_euler(x, v, dt, n, stream));
+}
+
+int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg, uint16_t* k_out, uint16_t* v_out,
+                  cudaStream_t stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || unit < 0) return WS_ERR_ARG;
+  if (seg != WS_SEG_COND && seg != WS_SEG_LATENT) return WS_ERR_ARG;
+  const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
+  if (n > 0) {
+    if (!k_out || !v_out) return WS_ERR_ARG;
+    if (!aligned16(k_out) || !aligned16(v_out)) return WS_ERR_ALIGN;
+  }
+  const int st = resident(h, unit);
+  if (st != WS_OK) return st;
+  const size_t slot = (size_t)(unit % h->C);
+  if (seg == WS_SEG_LATENT && !h->latent_ready[slot * h->cfg.n_layers + layer]) return WS_ERR_NOT_READY;
+  ReadParams p{};
+  p.cache = h->kv;
+  p.dst_k = k_out;
+  p.dst_v = v_out;
+  p.layer = layer;
+  p.n_tokens = n;
+  p.n_heads = h->cfg.n_heads;
+  p.head_dim = h->cfg.head_dim;
+  p.plane_rows = (int64_t)h->C * h->T;
+  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  return cuda_status(launch_read(p, stream));
+}
+
+int ws_cache_slot_table(const ws_cache_t* h, int64_t* slot_unit_host) {
+  if (!h || !slot_unit_host) return WS_ERR_ARG;
+  std::copy(h->slot_unit.begin(), h->slot_unit.end(), slot_unit_host);
+  return WS_OK;
+}
+
+int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info) {
+  if (!h || !info) return WS_ERR_ARG;
+  info->slots = h->C;
+  info->tokens_per_unit = h->T;
+  info->n_query = h->Nq;
+  info->newest_unit = h->newest;
+  info->cache_bytes = h->kv_bytes;
+  info->workspace_bytes = h->ws_bytes;
+  return WS_OK;
+}
+
+int ws_cache_set_splits(ws_cache_t* h, int n_split) {
+  if (!h || n_split < 0 || n_split > kMaxSplits) return WS_ERR_ARG;
+  h->force_splits = n_split;
+  return WS_OK;
+}
+
+int ws_sync(ws_cache_t* h, cudaStream_t stream) {
+  if (!h) return WS_ERR_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return WS_ERR_CUDA;
+  int s = 0;
+  if (cudaMemcpy(&s, h->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WS_ERR_CUDA;
+  if (s != 0) {
+    if (cudaMemset(h->d_status, 0, sizeof(int)) != cudaSuccess) return WS_ERR_CUDA;
+    return WS_ERR_DEVICE_TIMEOUT;
+  }
+  return WS_OK;
+}
+
+int ws_profile_enable(ws_cache_t* h, int enable) {
+  if (!h) return WS_ERR_ARG;
+  if (enable && !h->profiling) {
+    h->ev_attn.create(2048);
+    h->ev_comb.create(2048);
+    h->ev_lat.create(2048);
+  } else if (!enable && h->profiling) {
+    cudaDeviceSynchronize();
+    h->ev_attn.destroy();
+    h->ev_comb.destroy();
+    h->ev_lat.destroy();
+  }
+  h->profiling = enable != 0;
+  for (EventPool* e : {&h->ev_attn, &h->ev_comb, &h->ev_lat}) {
+    e->used = 0;
+    e->launches = 0;
+    e->ms = 0.0;
+  }
+  return WS_OK;
+}
+
+int ws_profile_read(ws_cache_t* h, ws_profile* out) {
+  if (!h || !out) return WS_ERR_ARG;
+  h->ev_attn.flush();
+  h->ev_comb.flush();
+  h->ev_lat.flush();
+  out->attention_launches = h->ev_attn.launches;
+  out->attention_ms = h->ev_attn.ms;
+  out->combine_launches = h->ev_comb.launches;
+  out->combine_ms = h->ev_comb.ms;
+  out->latent_write_launches = h->ev_lat.launches;
+  out->latent_write_ms = h->ev_lat.ms;
+  out->last_n_split = h->last_split;
+  out->last_ctas = h->last_ctas;
+  out->last_keys = h->last_keys;
+  return WS_OK;
+}
+
+}  // extern "C"
