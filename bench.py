@@ -19,7 +19,6 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -208,10 +207,11 @@ def run_ours(args, rank, local_rank, world):
     h = g.h
     next_unit = [w.unit]
 
-    def unit_step(x_dev, inputs=None, after_call=None, vel_of=None):
+    def unit_step(x_dev, inputs=None, after_call=None, vel_of=None, cond=None):
         """One unit: conditioning append, S x L attention calls with Euler updates, commit."""
         u = next_unit[0]
-        ws.ws_cache_append(h, u, ws.WS_SEG_COND, cond_k, cond_v)
+        ck, cv = (cond_k, cond_v) if cond is None else cond
+        ws.ws_cache_append(h, u, ws.WS_SEG_COND, ck, cv)
         for s in range(S):
             for l in range(L):
                 q, kn, vn = (q_all[s, l], kn_all[s, l], vn_all[s, l]) if inputs is None else inputs(s, l)
@@ -230,11 +230,13 @@ def run_ours(args, rank, local_rank, world):
     barrier(world, local_rank)
     torch.cuda.synchronize()
     with ClockSampler(local_rank) as clk:
+        torch.cuda.nvtx.range_push("timed")
         e0.record(stream)
         for _ in range(args.steps):
             unit_step(x)
         e1.record(stream)
         torch.cuda.synchronize()
+        torch.cuda.nvtx.range_pop()
     barrier(world, local_rank)
     step_ms = e0.elapsed_time(e1) / args.steps
     prof = ws.ws_profile_read(h)
@@ -261,7 +263,8 @@ def run_ours(args, rank, local_rank, world):
     extra = hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit)
 
     # ---- end to end: the same unit step with inputs copied from pinned host memory each step
-    e2e = run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, world, local_rank, flops_unit)
+    e2e = run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, (cond_k, cond_v), world,
+                  local_rank, flops_unit)
 
     clocks = clk.summary()
     g.close()
@@ -331,7 +334,8 @@ def hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, co
     }
 
 
-def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, world, local_rank, flops_unit):
+def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, cond, world, local_rank,
+            flops_unit):
     """Same unit step, each step's inputs copied host->device from pinned memory on a
     copy stream (double-buffered per layer-step) and the final latent copied back."""
     L, S = w.n_layers, w.steps
@@ -346,6 +350,8 @@ def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, 
     host_vel = vel.cpu().pin_memory()
     host_x = x0.cpu().pin_memory()
     host_x_out = torch.empty_like(host_x).pin_memory()
+    host_ck, host_cv = cond[0].cpu().pin_memory(), cond[1].cpu().pin_memory()
+    dck, dcv = torch.empty_like(cond[0]), torch.empty_like(cond[1])
     dbuf = torch.empty((2, 3) + tuple(qs), dtype=torch.bfloat16, device=dev)
     dvel = torch.empty_like(vel)
     x = torch.empty_like(x0)
@@ -359,6 +365,8 @@ def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, 
         with torch.cuda.stream(copy):
             x.copy_(host_x, non_blocking=True)
             dvel.copy_(host_vel, non_blocking=True)
+            dck.copy_(host_ck, non_blocking=True)
+            dcv.copy_(host_cv, non_blocking=True)
             first = torch.cuda.Event()
             first.record(copy)
 
@@ -385,7 +393,7 @@ def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, 
         def after_call(s, l):
             free[pos[(s, l)] % 2].record(comp)
 
-        unit_step(x, inputs, after_call, lambda s: dvel[s])
+        unit_step(x, inputs, after_call, lambda s: dvel[s], (dck, dcv))
         host_x_out.copy_(x, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -400,26 +408,30 @@ def run_e2e(args, ws, w, torch, dev, unit_step, q_all, kn_all, vn_all, vel, x0, 
     torch.cuda.synchronize()
     barrier(world, local_rank)
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world, dev)
-    h2d = (L * S * 3 * q_all[0, 0].numel() + vel.numel() + x0.numel()) * 2
+    h2d = (L * S * 3 * q_all[0, 0].numel() + vel.numel() + x0.numel() + 2 * cond[0].numel()) * 2
     d2h = x0.numel() * 2
     return {"value": round(aggregate(flops_unit, world, ms / 1e3, 1), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "note": "conditioning and commit K/V stay device-resident; q, k_new, v_new, velocities and x cross PCIe"}
+            "note": "per step, q/k_new/v_new of all 160 layer-steps, the conditioning slice, velocities and x "
+                    "are copied from pinned host memory; the committed latent K/V is produced on the device"}
 
 
 # ------------------------------------------------------- the oracle arm --
 
+_ORACLE = {}
+
+
 def oracle_sample(target_s: float, max_rows=None):
     """Time the fp64 oracle on a bounded sample of the same workload: one head of one
-    layer-step, as many query rows as fit in about target_s seconds."""
+    layer-step (layer 17, Euler step 1), as many query rows as fit in about target_s
+    seconds.  Input generation is not timed."""
     sys.path.insert(0, os.path.join(ROOT, "tests"))
-    import numpy as np
-
     from kv_cache_serving_ws_b200.workloads import FULL
     from oracle_side import oracle_cache
     w = FULL
-    cache, q, kn, vn = oracle_cache(w, 17, [0], 1)
-    # probe a few rows, then size the sample
+    if "case" not in _ORACLE:
+        _ORACLE["case"] = oracle_cache(w, 17, [0], 1)
+    cache, q, kn, vn = _ORACLE["case"]
     t0 = time.perf_counter()
     st, _ = cache.unit_attention(0, w.unit, q, kn, vn, rows=[0, 1])
     t_row = (time.perf_counter() - t0) / 2
@@ -436,10 +448,10 @@ def oracle_sample(target_s: float, max_rows=None):
         cores = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
     except Exception:
         cores = os.cpu_count() or 1
+    per_unit_ms = dt * w.n_heads * (w.n_query / rows) * w.n_layers * w.steps * 1e3
     return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"1 head x {rows} query rows of one layer-step of {w.name} ({w.n_keys} keys), "
-                      f"{dt:.1f} s; ms per unit extrapolated x{w.n_heads} heads x{w.n_query/rows:.2f} rows "
-                      f"x{w.n_layers * w.steps} layer-steps = {dt * w.n_heads * (w.n_query / rows) * w.n_layers * w.steps * 1e3:.0f} ms",
+            "sample": f"1 head x {rows} query rows of one layer-step of {w.name} ({w.n_keys} keys) in {dt:.1f} s; "
+                      f"a whole unit extrapolates to {per_unit_ms / 1e3:.0f} s",
             "seconds": round(dt, 2)}
 
 
@@ -467,6 +479,35 @@ def run_reference(args):
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(args):
+    """A single workload's attention calls, for profiler captures: prefill the
+    history, then `calls` attention calls of layer 0 of the current unit."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200.workloads import ALL, GpuSession
+    w = {"tiny": "tiny-192x336-5units-8x64", "v01": "v01-192x336-hist16-40x128", "v02": "v02-640x368-hist32-40x128",
+         "ring": "v02-640x368-ring128-u1000-40x128"}.get(args.case, args.case)
+    w = ALL[w]
+    g = GpuSession(w)
+    g.prefill()
+    q, kn, vn = g.step_inputs(0)
+    out = torch.empty_like(q)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(args.calls):
+        ws.ws_unit_attention(g.h, 0, w.unit, q, kn, vn, out)
+    e1.record()
+    st = ws.ws_sync(g.h, check=False)
+    ms = e0.elapsed_time(e1) / max(1, args.calls)
+    print(json.dumps({"case": w.name, "calls": args.calls, "ms_per_call": round(ms, 4),
+                      "TFLOP/s": round(w.flops_per_call() / ms / 1e9, 1), "status": ws.status_string(st)}))
+    g.close()
+    if st != ws.WS_OK:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -474,9 +515,14 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-baseline-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=5.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--case", default=None, help="profiling mode: tiny|v01|v02|ring (attention calls only)")
+    ap.add_argument("--calls", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        run_case(args)
+        return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     rank, local_rank, world = dist_env()

@@ -177,9 +177,13 @@ typedef struct {
 int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info);
 
 /*
- * ws_cache_set_splits -- number of key-range splits of each attention call
- * (split-K partials merged by a second kernel).  0 = automatic (chosen to fill
- * the 148 SMs), 1..16 forces that count (clamped to the number of key tiles).
+ * ws_cache_set_splits -- work decomposition of each attention call.  The
+ * attention kernel is persistent: one lane of CTAs per pair of 128-row query
+ * tiles; the CTAs of a lane share out its (head, key tile) iterations in equal
+ * contiguous ranges, and the heads whose range is cut between two CTAs are
+ * merged from fp32 partials by a second kernel.  n_split = CTAs per lane:
+ * 0 = automatic (one CTA per SM over all lanes), 1..1024 forces that count
+ * (reduced if the partials would not fit the workspace).
  */
 int ws_cache_set_splits(ws_cache_t* h, int n_split);
 
@@ -206,7 +210,7 @@ typedef struct {
   double combine_ms;
   int64_t latent_write_launches;
   double latent_write_ms;
-  int32_t last_n_split;        /* split count of the last attention call */
+  int32_t last_n_split;        /* CTAs per query-pair lane of the last attention call */
   int32_t last_ctas;           /* CTAs of the last attention launch */
   int64_t last_keys;           /* visible keys of the last attention call */
 } ws_profile;

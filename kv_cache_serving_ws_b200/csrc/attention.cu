@@ -11,20 +11,24 @@
 // that are not visible are never loaded (whole-unit skipping), and the last
 // tile of each run masks the rows past its end.
 //
-// One CTA computes a 128-row query tile of one head over one range of key tiles:
-//   warps 0-3  softmax: one query row per thread (= one TMEM lane), fp32 online
-//              softmax in base 2, P rounded to bf16 into swizzled shared memory,
-//              rescale of the O accumulator in TMEM when the running max moves
-//              by more than 2^8, epilogue;
-//   warp 4     TMA producer: Q once, then K and V tiles (2 stages each);
-//   warp 5     MMA issuer: S = Q K^T into one of two TMEM buffers, O += P V.
-// With several key ranges per (tile, head) the CTAs write fp32 partials (O, max,
-// sum) and a second kernel merges them by their log-sum-exp weights.
+// Persistent kernel, one CTA per SM, stream-K style: every CTA gets the same
+// number of (Q tile, head, key tile) iterations (see Decomp).  A CTA works on one
+// 128-row query tile of one head at a time:
+//   warps 0-3  softmax: one query row per thread (= one TMEM lane); fp32 online
+//              softmax in base 2 with a lazily moved reference max; P is rounded
+//              to bf16 and written back into the TMEM columns of its own S (A
+//              operand of the P.V product); epilogue of each item;
+//   warp 4     TMA producer: the Q tile of each item, K and V tiles (2 stages);
+//   warp 5     MMA issuer: S(j+1) = Q K(j+1)^T into the other of two TMEM S
+//              buffers before O += P(j) V(j) (A from TMEM, V as an MN-major B
+//              operand), so the next tile's QK^T overlaps this tile's softmax.
+// TMEM: S buffers [0,128) and [128,256), O [256, 256+D).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdio>
+#include <cstdlib>
 
 #include "kernels.cuh"
 #include "sm100.cuh"
@@ -35,48 +39,85 @@ namespace {
 
 enum Bar : int {
   kQFull = 0,
-  kKFull = 1,   // +stage
-  kKEmpty = 3,  // +stage
-  kVFull = 5,   // +stage
-  kVEmpty = 7,  // +stage
-  kSFull = 9,   // +buffer
-  kSEmpty = 11, // +buffer
-  kPFull = 13,
+  kQEmpty = 1,
+  kKFull = 2,    // +stage
+  kKEmpty = 4,   // +stage
+  kVFull = 6,    // +stage
+  kVEmpty = 8,   // +stage
+  kSFull = 10,   // +S buffer
+  kPFull = 12,   // +S buffer
   kPVDone = 14,
-  kMmaDone = 15,
-  kNumBars = 16
+  kOFull = 15,
+  kOFree = 16,
+  kMmaDone = 17,
+  kNumBars = 18
 };
 
-constexpr int kThreads = 192;
-constexpr int kTmemCols = 512;   // S buffers at columns [0,128) and [128,256), O at [256, 256+D)
+constexpr int kSoftmaxWarps = 4;
+constexpr int kProducerWarp = kSoftmaxWarps;
+constexpr int kMmaWarp = kSoftmaxWarps + 1;
+constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kTmemCols = 512;
 constexpr int kRowBytes = 128;   // one 128-byte swizzle row = 64 bf16
 
 template <int D>
 struct Smem {
   static constexpr int kChunks = D / 64;
-  static constexpr int kQBytes = kBlockM * D * 2;
+  static constexpr int kQTileBytes = kBlockM * D * 2;
   static constexpr int kTileBytes = kBlockN * D * 2;
-  static constexpr int kPBytes = kBlockM * kBlockN * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffK = kOffQ + kQTileBytes;
   static constexpr int kOffV = kOffK + 2 * kTileBytes;
-  static constexpr int kOffP = kOffV + 2 * kTileBytes;
-  static constexpr int kOffBar = kOffP + kPBytes;
+  static constexpr int kOffBar = kOffV + 2 * kTileBytes;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kBytes = kOffMisc + 64;
-  // One CTA per SM: its 512 TMEM columns are the whole TMEM of the SM.
+  // one CTA per SM: its 512 TMEM columns are all of the SM's TMEM
   static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
 };
 
-__device__ __forceinline__ void tile_info(const KeyRuns& r, int t, int& row0, int& valid) {
+__device__ __forceinline__ uint32_t tmem_s(uint32_t base, int b) { return base + (uint32_t)(b * 128); }
+__device__ __forceinline__ uint32_t tmem_o(uint32_t base) { return base + 256u; }
+
+__device__ __forceinline__ int tile_run(const KeyRuns& r, int t) {
   int k = 0, hi = r.n_runs - 1;          // last run with tile_begin <= t
   while (k < hi) {
     const int mid = (k + hi + 1) >> 1;
     if (r.tile_begin[mid] <= t) k = mid; else hi = mid - 1;
   }
-  const int local = t - r.tile_begin[k];
-  row0 = r.row_begin[k] + local * kBlockN;
-  valid = min(kBlockN, r.rows[k] - local * kBlockN);
+  return k;
+}
+__device__ __forceinline__ int tile_row0(const KeyRuns& r, int t) {
+  const int k = tile_run(r, t);
+  return r.row_begin[k] + (t - r.tile_begin[k]) * kBlockN;
+}
+__device__ __forceinline__ int tile_valid(const KeyRuns& r, int t) {
+  const int k = tile_run(r, t);
+  return min(kBlockN, r.rows[k] - (t - r.tile_begin[k]) * kBlockN);
+}
+
+// Position of the CTA-local iteration g: Q tile, head, key tile, item ordinal
+// within the CTA, and whether g opens / closes its item.
+struct Iter {
+  int qt, h, t, n;
+  bool first, last;
+};
+struct Range {
+  int lane, idx, gq;        // lane, CTA index in the lane, Q tiles of the lane
+  long long start;          // first lane iteration
+  int len;                  // iterations of this CTA
+  long long item0;          // lane-local item of the first iteration
+};
+__device__ __forceinline__ Iter iter_at(const Decomp& d, const Range& r, int g) {
+  const long long pos = r.start + g;
+  const long long item = pos / d.tiles;
+  Iter it;
+  it.t = (int)(pos - item * d.tiles);
+  it.h = (int)(item / r.gq);
+  it.qt = r.lane * d.group + (int)(item - (long long)it.h * r.gq);
+  it.n = (int)(item - r.item0);
+  it.first = (g == 0) || (it.t == 0);
+  it.last = (g == r.len - 1) || (it.t == d.tiles - 1);
+  return it;
 }
 
 // Bounded wait used only to drain in-flight copies and MMAs on the way out.
@@ -94,49 +135,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     unit_attention_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap kv_map,
                           const __grid_constant__ AttnParams p) {
   using S = Smem<D>;
+  const Decomp& d = p.dec;
+  Range rg;
+  rg.lane = blockIdx.x / d.lane_ctas;
+  rg.idx = blockIdx.x - rg.lane * d.lane_ctas;
+  rg.gq = lane_qtiles(d, rg.lane);
+  {
+    const long long per = lane_per(d, rg.lane);
+    const long long work = lane_work(d, rg.lane);
+    rg.start = (long long)rg.idx * per;
+    const long long end = rg.start + per < work ? rg.start + per : work;
+    rg.len = end > rg.start ? (int)(end - rg.start) : 0;
+    rg.item0 = rg.start / d.tiles;
+  }
+  if (rg.len == 0) return;                 // whole CTA: nothing allocated yet
+
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   uint8_t* sQ = smem + S::kOffQ;
   uint8_t* sK = smem + S::kOffK;
   uint8_t* sV = smem + S::kOffV;
-  uint8_t* sP = smem + S::kOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x % p.n_qtiles;
-  const int rest = blockIdx.x / p.n_qtiles;
-  const int split = rest % p.n_split;
-  const int h = rest / p.n_split;
-  const int t_begin = split * p.tiles_per_split;
-  const int t_end = min(p.runs.total_tiles, t_begin + p.tiles_per_split);
-  const int n_tiles = t_end - t_begin;
-  const int q0 = qt * kBlockM;
+  const int len = rg.len;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[kQFull], 1);
+    mbar_init(&bars[kQEmpty], 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kKFull + s], 1);
       mbar_init(&bars[kKEmpty + s], 1);
       mbar_init(&bars[kVFull + s], 1);
       mbar_init(&bars[kVEmpty + s], 1);
       mbar_init(&bars[kSFull + s], 1);
-      mbar_init(&bars[kSEmpty + s], 4);
+      mbar_init(&bars[kPFull + s], 4);
     }
-    mbar_init(&bars[kPFull], 4);
     mbar_init(&bars[kPVDone], 1);
+    mbar_init(&bars[kOFull], 1);
+    mbar_init(&bars[kOFree], 4);
     mbar_init(&bars[kMmaDone], 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&q_map);
     prefetch_tensormap(&kv_map);
   }
@@ -146,249 +196,271 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bars[kQFull], S::kQBytes);
-      for (int c = 0; c < S::kChunks; ++c)
-        tma_load_3d(sQ + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, h, q0);
-      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1};
+      int last_k[2] = {-1, -1}, last_v[2] = {-1, -1}, last_q = -1;
       bool ok = true;
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int s = i & 1;
-        const uint32_t use = (uint32_t)i >> 1;
-        int row0, valid;
-        tile_info(p.runs, t_begin + i, row0, valid);
+      for (int g = 0; g < len && ok; ++g) {
+        const Iter it = iter_at(d, rg, g);
+        if (it.first) {
+          if (it.n > 0 && !wait_phase(&bars[kQEmpty], (uint32_t)(it.n - 1) & 1, guard)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[kQFull], S::kQTileBytes);
+          for (int c = 0; c < S::kChunks; ++c)
+            tma_load_3d(sQ + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h, it.qt * kBlockM);
+          last_q = it.n;
+        }
+        const int s = g & 1;
+        const uint32_t use = (uint32_t)g >> 1;
+        const int row0 = tile_row0(p.runs, it.t);
         if (use > 0 && !wait_phase(&bars[kKEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars[kKFull + s], S::kTileBytes);
         for (int c = 0; c < S::kChunks; ++c)
           tma_load_3d(sK + s * S::kTileBytes + c * kBlockN * kRowBytes, &kv_map, &bars[kKFull + s], c * 64, row0,
-                      p.plane_k + h);
-        last_k[s] = i;
+                      p.plane_k + it.h);
+        last_k[s] = g;
         if (use > 0 && !wait_phase(&bars[kVEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
-        if (i != p.debug_skip_v_tile) {
+        if (g != p.debug_skip_v_tile) {
           mbar_arrive_expect_tx(&bars[kVFull + s], S::kTileBytes);
           for (int c = 0; c < S::kChunks; ++c)
             tma_load_3d(sV + s * S::kTileBytes + c * kBlockN * kRowBytes, &kv_map, &bars[kVFull + s], c * 64,
-                        row0, p.plane_v + h);
-          last_v[s] = i;
+                        row0, p.plane_v + it.h);
+          last_v[s] = g;
         }
       }
       if (!ok || *abort_flag) {
         // leaving early: let every copy already issued land before the CTA exits
-        drain_wait(&bars[kQFull], 0, p.timeout_ns);
+        if (last_q >= 0) drain_wait(&bars[kQFull], (uint32_t)last_q & 1, p.timeout_ns);
         for (int s = 0; s < 2; ++s) {
           if (last_k[s] >= 0) drain_wait(&bars[kKFull + s], ((uint32_t)last_k[s] >> 1) & 1, p.timeout_ns);
           if (last_v[s] >= 0) drain_wait(&bars[kVFull + s], ((uint32_t)last_v[s] >> 1) & 1, p.timeout_ns);
         }
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32(kBlockM, D, false, true);
-      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV), p_base = smem_u32(sP);
-      bool ok = wait_phase(&bars[kQFull], 0, guard);
-      for (int i = 0; ok && i <= n_tiles; ++i) {
-        if (i < n_tiles) {
-          const int s = i & 1;
-          if (!wait_phase(&bars[kKFull + s], ((uint32_t)i >> 1) & 1, guard)) break;
-          if (i >= 2 && !wait_phase(&bars[kSEmpty + s], ((uint32_t)(i - 2) >> 1) & 1, guard)) break;
-          tc_fence_after_sync();
-          const uint32_t d_tmem = tmem + (uint32_t)(s * kBlockN);
+      const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
+      // S(g) = Q K(g)^T into S buffer g % 2
+      auto issue_s = [&](int g) -> bool {
+        const Iter it = iter_at(d, rg, g);
+        const int s = g & 1;
+        if (it.first && !wait_phase(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
+        if (!wait_phase(&bars[kKFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_s(tmem, s);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (uint32_t)((kk >> 2) * kBlockM * kRowBytes + (kk & 3) * 32);
-            const uint32_t koff = (uint32_t)((kk >> 2) * kBlockN * kRowBytes + (kk & 3) * 32);
-            const uint64_t a = umma_smem_desc_sw128(q_base + off, 16, 1024);
-            const uint64_t b = umma_smem_desc_sw128(k_base + s * S::kTileBytes + koff, 16, 1024);
-            umma_bf16_ss(d_tmem, a, b, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&bars[kKEmpty + s]);
-          umma_commit(&bars[kSFull + s]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (uint32_t)((kk >> 2) * kBlockM * kRowBytes + (kk & 3) * 32);
+          const uint32_t koff = (uint32_t)((kk >> 2) * kBlockN * kRowBytes + (kk & 3) * 32);
+          const uint64_t da = umma_smem_desc_sw128(q_base + off, 16, 1024);
+          const uint64_t db = umma_smem_desc_sw128(k_base + s * S::kTileBytes + koff, 16, 1024);
+          umma_bf16_ss(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
         }
-        if (i >= 1) {
-          const int j = i - 1;
-          const int s = j & 1;
-          if (!wait_phase(&bars[kPFull], (uint32_t)j & 1, guard)) break;
-          if (!wait_phase(&bars[kVFull + s], ((uint32_t)j >> 1) & 1, guard)) break;
-          tc_fence_after_sync();
-          const uint32_t o_tmem = tmem + 2 * kBlockN;
+        umma_commit(&bars[kSFull + s]);
+        umma_commit(&bars[kKEmpty + s]);
+        if (it.last) umma_commit(&bars[kQEmpty]);
+        return true;
+      };
+      // O += P(g) V(g), P(g) in the TMEM columns of S buffer g % 2
+      auto issue_pv = [&](int g) -> bool {
+        const Iter it = iter_at(d, rg, g);
+        const int s = g & 1;
+        if (!wait_phase(&bars[kVFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
+        if (!wait_phase(&bars[kPFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
+        if (it.first && it.n > 0 && !wait_phase(&bars[kOFree], (uint32_t)(it.n - 1) & 1, guard)) return false;
+        tc_fence_after_sync();
+        const uint32_t o_tmem = tmem_o(tmem);
+        const uint32_t p_tmem = tmem_s(tmem, s);
 #pragma unroll
-          for (int kk = 0; kk < kBlockN / 16; ++kk) {
-            const uint32_t poff = (uint32_t)((kk >> 2) * kBlockM * kRowBytes + (kk & 3) * 32);
-            const uint64_t a = umma_smem_desc_sw128(p_base + poff, 16, 1024);
-            // V tile: MN-major B operand; 16 keys = 16 rows of 128 bytes; the next
-            // 64 head-dim columns sit one chunk (kBlockN rows) further.
-            const uint64_t b = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
-                                                    kBlockN * kRowBytes, 1024);
-            umma_bf16_ss(o_tmem, a, b, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(&bars[kVEmpty + s]);
-          umma_commit(&bars[kPVDone]);
+        for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          // 16 keys = 8 TMEM columns of packed bf16 pairs; V: 16 rows of 128 bytes,
+          // the next 64 head-dim columns one chunk (kBlockN rows) further
+          const uint64_t db = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
+                                                   kBlockN * kRowBytes, 1024);
+          umma_bf16_ts(o_tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
         }
+        umma_commit(&bars[kPVDone]);
+        umma_commit(&bars[kVEmpty + s]);
+        if (it.last) umma_commit(&bars[kOFull]);
+        return true;
+      };
+      bool ok = issue_s(0);
+      for (int g = 0; ok && g < len; ++g) {
+        if (g + 1 < len) ok = issue_s(g + 1);
+        if (ok) ok = issue_pv(g);
       }
       umma_commit(&bars[kMmaDone]);
       drain_wait(&bars[kMmaDone], 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int row = threadIdx.x;  // TMEM lane
+    const int row = threadIdx.x;             // TMEM lane
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem + lane_base;
-    const uint32_t t_o = tmem + lane_base + 2 * kBlockN;
+    const uint32_t t_o = tmem_o(tmem) + lane_base;
     float m_ref = -INFINITY;  // reference max of this row, log2 units
     float l_sum = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      const int s = j & 1;
-      ok = wait_phase(&bars[kSFull + s], ((uint32_t)j >> 1) & 1, guard);
+    for (int g = 0; g < len; ++g) {
+      const Iter it = iter_at(d, rg, g);
+      const int b = g & 1;
+      const uint32_t t_s = tmem_s(tmem, b) + lane_base;
+      if (it.first) {
+        m_ref = -INFINITY;
+        l_sum = 0.f;
+      }
+      ok = wait_phase(&bars[kSFull + b], ((uint32_t)g >> 1) & 1, guard);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after_sync();
       uint32_t sr[kBlockN];
-      tmem_load_128(t_s + (uint32_t)(s * kBlockN), sr);
-      tc_fence_before_sync();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kSEmpty + s]);
-
-      int row0, valid;
-      tile_info(p.runs, t_begin + j, row0, valid);
-      float mx = -INFINITY;
+      tmem_load_128(t_s, sr);
+      const int valid = tile_valid(p.runs, it.t);
+      if (valid < kBlockN) {
 #pragma unroll
-      for (int c = 0; c < kBlockN; ++c) {
-        float v = __uint_as_float(sr[c]);
-        if (c >= valid) v = -INFINITY;
-        sr[c] = __float_as_uint(v);
-        mx = fmaxf(mx, v);
+        for (int c = 0; c < kBlockN; ++c)
+          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
-      const float m_cand = mx * p.scale_log2;
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+#pragma unroll
+      for (int c = 8; c < kBlockN; c += 8)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[c + k]));
+      const float m_cand =
+          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
+          p.scale_log2;
+      // Move the reference max only when P would exceed 2^8 (or for a new item).
+      const bool move = it.first || m_cand > m_ref + 8.f;
       float alpha = 1.f;
-      bool rescale = false;
-      if (m_cand > m_ref + 8.f) {
+      if (move) {
         alpha = ex2_approx(m_ref - m_cand);
         l_sum *= alpha;
         m_ref = m_cand;
-        rescale = true;
       }
       const float neg_m = -m_ref;
-      float rs = 0.f;
-      uint32_t packed[kBlockN / 2];
+      float rs[8];
 #pragma unroll
-      for (int c = 0; c < kBlockN / 2; ++c) {
-        const float a = ex2_approx(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m));
-        const float b = ex2_approx(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, neg_m));
-        rs += a + b;
-        packed[c] = pack_bf16x2(a, b);
-      }
-      l_sum += rs;
-
-      if (j > 0) {
-        // the previous P.V has finished: the P buffer is free and O is stable
-        ok = wait_phase(&bars[kPVDone], (uint32_t)(j - 1) & 1, guard);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-        tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, rescale)) {
+      for (int k = 0; k < 8; ++k) rs[k] = 0.f;
+      uint32_t pk[kBlockN / 2];
 #pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            tmem_load_32(t_o + (uint32_t)c, o);
+      for (int c = 0; c < kBlockN; c += 16) {
 #pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_store_32(t_o + (uint32_t)c, o);
-          }
+        for (int k = 0; k < 8; ++k) {
+          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[c + 2 * k]), p.scale_log2, neg_m));
+          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[c + 2 * k + 1]), p.scale_log2, neg_m));
+          rs[k] += e0 + e1;
+          pk[c / 2 + k] = pack_bf16x2(e0, e1);
         }
       }
-      // P row -> shared memory, K-major with the 128-byte swizzle: 16-byte piece
-      // `pc` of a 128-byte row lands at position pc ^ (row & 7).
-#pragma unroll
-      for (int c16 = 0; c16 < kBlockN / 8; ++c16) {
-        const int chunk = c16 >> 3, piece = c16 & 7;
-        uint8_t* dst = sP + chunk * kBlockM * kRowBytes + row * kRowBytes + ((piece ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) =
-            make_uint4(packed[4 * c16], packed[4 * c16 + 1], packed[4 * c16 + 2], packed[4 * c16 + 3]);
+      l_sum += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+      tmem_store_64(t_s, pk);                // keys 2c, 2c+1 -> column c of the S buffer
+      if (g > 0) {
+        // O holds P(g-1) V(g-1) once this completes; needed before rescaling it
+        ok = wait_phase(&bars[kPVDone], (uint32_t)(g - 1) & 1, guard);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       }
-      fence_proxy_async_smem();
+      if (__any_sync(0xffffffffu, move && !it.first)) {
+        tc_fence_after_sync();
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          tmem_load_32(t_o + (uint32_t)c, o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+          tmem_store_32(t_o + (uint32_t)c, o);
+        }
+      }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kPFull]);
-    }
+      if (lane == 0) mbar_arrive(&bars[kPFull + b]);
 
-    if (ok) {
-      ok = wait_phase(&bars[kPVDone], (uint32_t)(n_tiles - 1) & 1, guard);
-      ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
-      tc_fence_after_sync();
-      const int q_row = q0 + row;
-      if (p.n_split == 1) {
+      if (it.last) {
+        // ---- epilogue of the item (qt, h)
+        ok = wait_phase(&bars[kOFull], (uint32_t)it.n & 1, guard);
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after_sync();
+        const int q_row = it.qt * kBlockM + row;
+        int c_first, pieces;
+        item_span(d, it.qt, it.h, c_first, pieces);
         const float inv = 1.f / l_sum;
-        uint16_t* dst = p.out + ((size_t)q_row * p.n_heads + h) * D;
-#pragma unroll
+        uint16_t* dst = p.out + ((size_t)q_row * p.n_heads + it.h) * D;
+        size_t prow = 0;
+        if (pieces > 1) {
+          const size_t slot = ((size_t)it.qt * p.n_heads + it.h) * d.max_pieces + (size_t)(rg.idx - c_first);
+          prow = slot * kBlockM + (size_t)row;
+          *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
+        }
+        // O in 32-column chunks: bf16 output of a whole item, fp32 partial otherwise
+#pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
           tmem_load_32(t_o + (uint32_t)c, o);
-          if (q_row < p.n_query) {
+          if (pieces == 1) {
+            if (q_row < p.n_query) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
-              *reinterpret_cast<uint4*>(dst + c + 8 * k) = w;
+              for (int k = 0; k < 32; k += 8) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
+                w.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+                w.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
+                w.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
+                *reinterpret_cast<uint4*>(dst + c + k) = w;
+              }
             }
+          } else {
+            float* po = p.part_o + prow * D + c;
+#pragma unroll
+            for (int k = 0; k < 32; k += 4)
+              *reinterpret_cast<uint4*>(po + k) = make_uint4(o[k], o[k + 1], o[k + 2], o[k + 3]);
           }
         }
-      } else {
-        const size_t rows_pad = (size_t)p.n_qtiles * kBlockM;
-        const size_t base = ((size_t)split * p.n_heads + h) * rows_pad + (size_t)q_row;
-        float* po = p.part_o + base * D;
-#pragma unroll
-        for (int c = 0; c < D; c += 32) {
-          uint32_t o[32];
-          tmem_load_32(t_o + (uint32_t)c, o);
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            *reinterpret_cast<uint4*>(po + c + 4 * k) = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
-        }
-        *reinterpret_cast<float2*>(p.part_ml + base * 2) = make_float2(m_ref, l_sum);
+        tc_fence_before_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[kOFree]);
       }
     }
   }
 
   tc_fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// Merge of the split-K partials: out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
+// Merge of the partials of an item cut between CTAs:
+//   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
 // One warp per (row, head); each lane owns D/32 consecutive columns.
 template <int D>
-__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ AttnParams p) {
   constexpr int kPer = D / 32;
   const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   if (gw >= p.n_query * p.n_heads) return;
   const int row = gw / p.n_heads;
   const int h = gw - row * p.n_heads;
-  const size_t rows_pad = (size_t)p.n_qtiles * kBlockM;
+  const int qt = row / kBlockM;
+  int c_first, pieces;
+  item_span(p.dec, qt, h, c_first, pieces);
+  if (pieces == 1) return;                       // written directly by its CTA
+  const size_t slot0 = ((size_t)qt * p.n_heads + h) * p.dec.max_pieces;
+  const int r = row - qt * kBlockM;
   float m_all = -INFINITY;
-  for (int s = 0; s < p.n_split; ++s)
-    m_all = fmaxf(m_all, p.part_ml[(((size_t)s * p.n_heads + h) * rows_pad + row) * 2]);
+  for (int k = 0; k < pieces; ++k) m_all = fmaxf(m_all, p.part_ml[((slot0 + k) * kBlockM + r) * 2]);
   float l_all = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  for (int s = 0; s < p.n_split; ++s) {
-    const size_t base = ((size_t)s * p.n_heads + h) * rows_pad + row;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + base * 2);
+  for (int k = 0; k < pieces; ++k) {
+    const size_t prow = (slot0 + k) * kBlockM + r;
+    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
     const float w = ex2_approx(ml.x - m_all);
     l_all += w * ml.y;
-    const float* po = p.part_o + base * D + lane * kPer;
+    const float* po = p.part_o + prow * D + lane * kPer;
     if constexpr (kPer == 4) {
       const float4 o = *reinterpret_cast<const float4*>(po);
       acc[0] += w * o.x; acc[1] += w * o.y; acc[2] += w * o.z; acc[3] += w * o.w;
@@ -461,10 +533,17 @@ static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMa
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const int grid = p.n_qtiles * p.n_heads * p.n_split;
+  const int grid = p.dec.lanes * p.dec.lane_ctas;
   if (ctas) *ctas = grid;
   unit_attention_kernel<D><<<grid, kThreads, Smem<D>::kAlloc, stream>>>(q_map, kv_map, p);
-  return cudaGetLastError();
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess && std::getenv("WS_DEBUG")) {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, unit_attention_kernel<D>);
+    std::fprintf(stderr, "ws: attention launch failed: %s (grid %d, block %d, smem %d; kernel regs %d, max threads %d)\n",
+                 cudaGetErrorString(e), grid, kThreads, Smem<D>::kAlloc, fa.numRegs, fa.maxThreadsPerBlock);
+  }
+  return e;
 }
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p, int head_dim,
@@ -474,13 +553,13 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
   return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_combine(const AttnParams& p, int head_dim, cudaStream_t stream) {
+cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
   const long long warps = (long long)p.n_query * p.n_heads;
   const int grid = (int)((warps * 32 + 255) / 256);
   if (head_dim == 128)
-    combine_kernel<128><<<grid, 256, 0, stream>>>(p);
+    merge_kernel<128><<<grid, 256, 0, stream>>>(p);
   else if (head_dim == 64)
-    combine_kernel<64><<<grid, 256, 0, stream>>>(p);
+    merge_kernel<64><<<grid, 256, 0, stream>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

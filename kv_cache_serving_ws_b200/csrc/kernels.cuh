@@ -6,36 +6,72 @@
 
 namespace ws {
 
-constexpr int kBlockM = 128;   // query rows per CTA (one TMEM lane each)
+constexpr int kBlockM = 128;   // query rows per Q tile (one TMEM lane each)
 constexpr int kBlockN = 128;   // keys per tile
 constexpr int kMaxRuns = 192;  // visible row runs per attention call (>= slots of any ring with gaps)
-constexpr int kMaxSplits = 16;
+constexpr int kMaxLaneCtas = 1024;
 
 // Visible key rows of one (layer, head) plane: runs of consecutive rows, cut
-// into kBlockN-row tiles; tile_begin[r] is the first global tile of run r.
+// into kBlockN-row tiles; tile_begin[r] is the first tile of run r.
 struct KeyRuns {
   int32_t n_runs;
-  int32_t total_tiles;
+  int32_t total_tiles;      // key tiles of one (Q tile, head) item
   int32_t row_begin[kMaxRuns];
   int32_t rows[kMaxRuns];
   int32_t tile_begin[kMaxRuns + 1];
 };
 
+// Work decomposition.  An item is (Q tile qt, head h) over all key tiles.  The
+// Q tiles are cut into lanes of `group` consecutive tiles; every lane has
+// `lane_ctas` CTAs, and CTA idx of a lane processes the iterations
+// [idx*per, (idx+1)*per) of its lane's (head, Q tile of the lane, key tile)
+// sequence, head major.  CTAs with the same idx in different lanes then read
+// the same K/V tiles at about the same time (L2 reuse).  An item covered by
+// one CTA is written as bf16 directly; an item cut between CTAs is written as
+// fp32 partials (slot item*max_pieces + piece, item = qt*H + h) and merged.
+struct Decomp {
+  int32_t n_qtiles;
+  int32_t group;            // Q tiles per lane
+  int32_t lanes;
+  int32_t lane_ctas;
+  int32_t tiles;            // key tiles per item
+  int32_t heads;
+  int32_t max_pieces;
+};
+
+__host__ __device__ inline int lane_qtiles(const Decomp& d, int lane) {
+  const int left = d.n_qtiles - lane * d.group;
+  return left < d.group ? left : d.group;
+}
+__host__ __device__ inline long long lane_work(const Decomp& d, int lane) {
+  return (long long)lane_qtiles(d, lane) * d.heads * d.tiles;
+}
+__host__ __device__ inline long long lane_per(const Decomp& d, int lane) {
+  return (lane_work(d, lane) + d.lane_ctas - 1) / d.lane_ctas;
+}
+// First lane iteration of item (qt, h) and the CTAs (lane-local) that cover it.
+__host__ __device__ inline void item_span(const Decomp& d, int qt, int h, int& first_cta, int& pieces) {
+  const int lane = qt / d.group;
+  const int a = qt - lane * d.group;
+  const long long start = ((long long)h * lane_qtiles(d, lane) + a) * d.tiles;
+  const long long per = lane_per(d, lane);
+  first_cta = (int)(start / per);
+  pieces = (int)((start + d.tiles - 1) / per) - first_cta + 1;
+}
+
 struct AttnParams {
   int32_t n_query;          // Nq
   int32_t n_heads;          // H
-  int32_t n_qtiles;         // ceil(Nq / kBlockM)
-  int32_t n_split;          // key-range splits (1 = write bf16 output directly)
-  int32_t tiles_per_split;
   int32_t plane_k;          // KV-map plane index of head 0's K of this layer
   int32_t plane_v;          // same for V
   float scale_log2;         // log2(e) / sqrt(D)
-  uint16_t* out;            // [Nq][H][D] bf16, when n_split == 1
-  float* part_o;            // [n_split][H][n_qtiles*kBlockM][D] fp32, when n_split > 1
-  float* part_ml;           // [n_split][H][n_qtiles*kBlockM][2]  (running max in log2 units, sum)
+  uint16_t* out;            // [Nq][H][D] bf16
+  float* part_o;            // [n_qtiles*H*max_pieces][kBlockM][D] fp32
+  float* part_ml;           // [n_qtiles*H*max_pieces][kBlockM][2] (reference max in log2 units, sum)
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
-  int32_t debug_skip_v_tile;  // test hook: never load V of this local tile (-1 = off)
+  int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)
+  Decomp dec;
   KeyRuns runs;
 };
 
@@ -46,7 +82,8 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
                              int head_dim, int* ctas, cudaStream_t stream);
-cudaError_t launch_combine(const AttnParams& p, int head_dim, cudaStream_t stream);
+// Merge of the partials of items shared by several CTAs (no-op for the others).
+cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream);
 
 // Copy a [L][n][H][D] token-major slice into the head-major cache planes:
 // plane (l*2 + kv)*H + h, rows row0 .. row0+n-1 of each plane.

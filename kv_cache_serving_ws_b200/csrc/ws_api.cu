@@ -60,7 +60,8 @@ struct ws_cache {
   size_t ws_bytes = 0;
   int* d_status = nullptr;
   CUtensorMap kv_map;
-  int force_splits = 0;
+  int force_lane_ctas = 0;
+  int64_t slot_cap = 0;
   uint64_t timeout_ns = 2000000000ull;
   int debug_skip_v_tile = -1;
   bool profiling = false;
@@ -124,29 +125,48 @@ int plan_runs(const ws_cache_config& cfg, const int64_t* slot_unit, const uint8_
   return WS_OK;
 }
 
-// Number of key-range splits: minimise (waves of CTAs) x (tiles per CTA + fixed
-// per-CTA cost) + the merge pass, over 1..kMaxSplits.
-int choose_splits(int base_ctas, int total_tiles, int head_dim, int forced) {
-  const int cap = std::min(kMaxSplits, std::max(1, total_tiles));
-  if (forced > 0) return std::min(forced, cap);
+// Work decomposition of one attention call (see Decomp in kernels.cuh).  The Q
+// tiles are grouped into lanes so that the lanes together hold one CTA per SM;
+// the group size minimises the iterations of the busiest CTA (ties: the
+// smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
+// iterations.  `forced` > 0 fixes the CTAs per lane.  Returns false when the
+// partial slots would not fit the workspace even with one CTA per lane.
+bool decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap) {
   const int sms = sm_count();
-  const double kFixedTiles = 3.0;                       // prologue + epilogue of one CTA, in tile times
-  const double tile_s = 0.8e-6, hbm = 6.5e12;          // rough tile time and HBM rate
-  int best = 1;
-  double best_cost = 1e300;
-  for (int n = 1; n <= cap; ++n) {
-    const int tps = (total_tiles + n - 1) / n;
-    const int n_eff = (total_tiles + tps - 1) / tps;
-    if (n_eff != n) continue;
-    const double waves = std::ceil((double)base_ctas * n / sms);
-    double cost = waves * (tps + kFixedTiles);
-    if (n > 1) cost += 5.0 + (double)n * base_ctas * kBlockM * head_dim * 4.0 / hbm / tile_s;
-    if (cost < best_cost - 1e-9) {
+  d.n_qtiles = n_qtiles;
+  d.heads = heads;
+  d.tiles = tiles;
+  int best_g = 1, best_cpl = 1;
+  long long best_cost = -1;
+  int prev_lanes = -1;
+  for (int g = 1; g <= n_qtiles; ++g) {
+    const int lanes = (n_qtiles + g - 1) / g;
+    if (lanes == prev_lanes) continue;
+    prev_lanes = lanes;
+    const long long work = (long long)g * heads * tiles;
+    long long cpl = forced > 0 ? forced : std::max(1, sms / lanes);
+    cpl = std::min<long long>(cpl, std::max<long long>(1, forced > 0 ? work : work / 2));
+    cpl = std::min<long long>(cpl, kMaxLaneCtas);
+    const long long cost = (work + cpl - 1) / cpl;
+    if (best_cost < 0 || cost < best_cost) {
       best_cost = cost;
-      best = n;
+      best_g = g;
+      best_cpl = (int)cpl;
     }
   }
-  return best;
+  d.group = best_g;
+  d.lanes = (n_qtiles + best_g - 1) / best_g;
+  for (int cpl = best_cpl;; cpl = std::max(1, cpl / 2)) {
+    d.lane_ctas = cpl;
+    long long min_per = -1;
+    for (int ln = 0; ln < d.lanes; ++ln) {
+      const long long per = lane_per(d, ln);
+      if (min_per < 0 || per < min_per) min_per = per;
+    }
+    d.max_pieces = (int)((tiles + min_per - 1) / min_per) + 1;
+    if ((int64_t)n_qtiles * heads * d.max_pieces <= slot_cap) return true;
+    if (cpl == 1) return false;
+  }
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WS_OK : WS_ERR_CUDA; }
@@ -208,9 +228,11 @@ int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t s
   const int L = cfg->n_layers, H = cfg->n_heads, D = cfg->head_dim;
   const int64_t rows = (int64_t)h->C * h->T;
   h->kv_bytes = (size_t)L * 2 * H * rows * D * 2;
-  const int64_t rows_pad = (int64_t)((h->Nq + kBlockM - 1) / kBlockM) * kBlockM;
-  const size_t part_o_bytes = (size_t)kMaxSplits * H * rows_pad * D * 4;
-  const size_t part_ml_bytes = (size_t)kMaxSplits * H * rows_pad * 2 * 4;
+  // partial slots: items x (ceil(SMs / H) + 1) bounds every automatic decomposition
+  const int64_t n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
+  h->slot_cap = n_qtiles * H * ((sm_count() + H - 1) / H + 1);
+  const size_t part_o_bytes = (size_t)h->slot_cap * kBlockM * D * 4;
+  const size_t part_ml_bytes = (size_t)h->slot_cap * kBlockM * 2 * 4;
   h->ws_bytes = part_o_bytes + part_ml_bytes;
   int st = WS_OK;
   if (cudaMalloc(&h->kv, h->kv_bytes) != cudaSuccess || cudaMalloc(&h->part_o, part_o_bytes) != cudaSuccess ||
@@ -337,10 +359,15 @@ int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q,
   // 2. attention (+ merge of split partials)
   p.n_query = h->Nq;
   p.n_heads = H;
-  p.n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
-  p.n_split = choose_splits(p.n_qtiles * H, tiles, D, h->force_splits);
-  p.tiles_per_split = (tiles + p.n_split - 1) / p.n_split;
-  p.n_split = (tiles + p.tiles_per_split - 1) / p.tiles_per_split;
+  const int n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
+  if (!decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas, h->slot_cap)) return WS_ERR_UNSUPPORTED;
+  bool any_split = false;
+  for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
+    for (int hh = 0; hh < H && !any_split; ++hh) {
+      int c_first, pieces;
+      item_span(p.dec, qt, hh, c_first, pieces);
+      any_split = pieces > 1;
+    }
   p.plane_k = (layer * 2 + 0) * H;
   p.plane_v = (layer * 2 + 1) * H;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
@@ -355,13 +382,13 @@ int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q,
   int ctas = 0;
   if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
-  if (p.n_split > 1) {
+  if (any_split) {
     ev = h->profiling ? h->ev_comb.next() : nullptr;
     if (ev) cudaEventRecord(ev[0], stream);
-    if (launch_combine(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
+    if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
     if (ev) cudaEventRecord(ev[1], stream);
   }
-  h->last_split = p.n_split;
+  h->last_split = p.dec.lane_ctas;
   h->last_ctas = ctas;
   h->last_keys = keys;
   return WS_OK;
@@ -419,8 +446,8 @@ int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info) {
 }
 
 int ws_cache_set_splits(ws_cache_t* h, int n_split) {
-  if (!h || n_split < 0 || n_split > kMaxSplits) return WS_ERR_ARG;
-  h->force_splits = n_split;
+  if (!h || n_split < 0 || n_split > kMaxLaneCtas) return WS_ERR_ARG;
+  h->force_lane_ctas = n_split;
   return WS_OK;
 }
 
@@ -439,9 +466,10 @@ int ws_sync(ws_cache_t* h, cudaStream_t stream) {
 int ws_profile_enable(ws_cache_t* h, int enable) {
   if (!h) return WS_ERR_ARG;
   if (enable && !h->profiling) {
-    h->ev_attn.create(2048);
-    h->ev_comb.create(2048);
-    h->ev_lat.create(2048);
+    // enough pairs for ~100 unit steps of 160 calls before a mid-run flush
+    h->ev_attn.create(16384);
+    h->ev_comb.create(16384);
+    h->ev_lat.create(16384);
   } else if (!enable && h->profiling) {
     cudaDeviceSynchronize();
     h->ev_attn.destroy();
