@@ -231,6 +231,36 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit,
                     const uint8_t* latent_ready, int layer, int64_t unit,
                     int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs);
 
+/*
+ * ws_attention_noalloc -- block-causal attention for callers that cannot
+ * allocate device memory.  The paper has no counterpart: this is an interface
+ * for callers that must not call cudaMalloc (inside a CUDA-graph capture that
+ * may hold no allocation, under a framework that owns every allocation and
+ * hands out only fixed buffers, or in a real-time loop that may not take the
+ * allocator's locks or fail on memory halfway through a unit).  Such callers
+ * cannot create a ws_cache, so this call takes caller-owned K/V planes and
+ * keeps its scratch (the fp32 partials of query tiles whose key range is cut
+ * between CTAs, and a status word) in a file-scope device array of 48 MiB that
+ * every device loading this part of the library holds until exit.
+ *
+ * For every head h and query row i:
+ *     out[i][h] = sum_j softmax_j(q[i][h] . k_j[h] / sqrt(D)) v_j[h],  0 <= j < n_keys
+ * q, out: [n_query][n_heads][head_dim]; kv: [2][n_heads][n_keys][head_dim], the K
+ * planes of all heads, then the V planes (the cache's per-layer layout); all
+ * caller-owned device memory, 16-byte aligned.  Same arithmetic as
+ * ws_unit_attention.
+ * The first call on a device looks up the array's device address (with that
+ * device current); make it before any stream capture.  Calls never allocate.
+ * All calls share the array and it keeps the last call's contents: calls that
+ * overlap on the GPU race on it, so the caller serialises them (one stream, or
+ * ordering between streams).  A kernel wait that runs out leaves its status in
+ * the array, which this call clears at its start and does not read back.
+ * Errors: WS_ERR_ARG, WS_ERR_ALIGN, WS_ERR_UNSUPPORTED (head_dim other than 64 or
+ * 128, or partials that would not fit the 48 MiB array), WS_ERR_CUDA.
+ */
+int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query,
+                         int32_t n_keys, int32_t n_heads, int32_t head_dim, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

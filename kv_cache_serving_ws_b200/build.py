@@ -24,7 +24,7 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "-c
          "--expt-relaxed-constexpr", "-I", INCLUDE]
 
 LIBS = {
-    "libws.so": ["ws_api.cu", "attention.cu", "copy_kernels.cu", "euler.cu"],
+    "libws.so": ["ws_api.cu", "attention.cu", "copy_kernels.cu", "euler.cu", "noalloc.cu"],
     "libws_synth.so": ["synth.cu"],
 }
 HEADERS = ["kernels.cuh", "sm100.cuh", "tmem_ldst.cuh"]

@@ -82,6 +82,9 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
                              int head_dim, int* ctas, cudaStream_t stream);
+// Chooses the work decomposition of one attention call (defined in ws_api.cu).
+bool decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap);
+
 // Merge of the partials of items shared by several CTAs (no-op for the others).
 cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream);
 

@@ -1,0 +1,117 @@
+// ws_attention_noalloc: the block-causal attention kernel for callers that
+// cannot allocate device memory.
+//
+// Who needs it: code that runs where cudaMalloc is unavailable or forbidden --
+// inside a CUDA-graph capture that must not contain allocation nodes, under a
+// host framework that owns every device allocation through its own pool and
+// hands out only fixed buffers, or in a real-time loop that may not take the
+// allocator's locks or risk an out-of-memory failure halfway through a 160 ms
+// unit.  Such a caller cannot create a ws_cache (which allocates the cache and
+// its workspace), so this entry point works on K/V planes the caller already
+// owns and keeps its own scratch -- the fp32 partials of query tiles whose key
+// range is cut between two CTAs, and the kernel's status word -- in one
+// file-scope device array instead of allocated memory.
+//
+// Limits and sharing: the array holds kScratchBytes (48 MiB) on every device
+// that loads this part of the library, until the process exits.  Requests
+// whose partials would not fit are rejected with WS_ERR_UNSUPPORTED.  All
+// calls share the array, and it keeps the last call's contents: calls that
+// overlap on the GPU (different streams, or different host threads without
+// ordering) race on it and must be serialised by the caller.  The status word
+// is cleared at the start of every call; the partials need no clearing,
+// because every slot the merge reads is written first by the same call.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/ws.h"
+#include "kernels.cuh"
+
+namespace {
+
+constexpr size_t kScratchBytes = size_t(48) << 20;
+constexpr size_t kStatusBytes = 256;            // the status word, padded to keep the partials aligned
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
+
+// Device address of g_scratch per device, looked up once with that device current.
+std::mutex g_setup_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+int scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WS_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (!g_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) return WS_ERR_CUDA;
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return WS_OK;
+}
+
+}  // namespace
+
+extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query,
+                                    int32_t n_keys, int32_t n_heads, int32_t head_dim, cudaStream_t stream) {
+  using namespace ws;
+  if (!q || !kv || !out || n_query < 1 || n_keys < 1 || n_heads < 1) return WS_ERR_ARG;
+  if (head_dim != 64 && head_dim != 128) return WS_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kv) | reinterpret_cast<uintptr_t>(out)) & 15u)
+    return WS_ERR_ALIGN;
+  if ((int64_t)n_heads * 2 >= ((int64_t)1 << 31)) return WS_ERR_ARG;
+
+  // one run of visible keys: rows [0, n_keys) of every plane
+  AttnParams p{};
+  p.runs.n_runs = 1;
+  p.runs.row_begin[0] = 0;
+  p.runs.rows[0] = n_keys;
+  p.runs.tile_begin[0] = 0;
+  p.runs.tile_begin[1] = (n_keys + kBlockN - 1) / kBlockN;
+  p.runs.total_tiles = p.runs.tile_begin[1];
+
+  // scratch layout: [status | part_ml | part_o]; slots sized for this call
+  const int n_qtiles = (n_query + kBlockM - 1) / kBlockM;
+  const size_t slot_bytes = (size_t)kBlockM * (head_dim + 2) * sizeof(float);
+  const int64_t slot_cap = (int64_t)((kScratchBytes - kStatusBytes) / slot_bytes);
+  if (!decompose(p.dec, n_qtiles, n_heads, p.runs.total_tiles, 0, slot_cap)) return WS_ERR_UNSUPPORTED;
+  const size_t slots = (size_t)n_qtiles * n_heads * p.dec.max_pieces;
+
+  void* base = nullptr;
+  const int st = scratch_address(&base);
+  if (st != WS_OK) return st;
+  unsigned char* b = static_cast<unsigned char*>(base);
+  p.status = reinterpret_cast<int*>(b);
+  p.part_ml = reinterpret_cast<float*>(b + kStatusBytes);
+  p.part_o = reinterpret_cast<float*>(b + kStatusBytes + slots * kBlockM * 2 * sizeof(float));
+
+  p.n_query = n_query;
+  p.n_heads = n_heads;
+  p.plane_k = 0;
+  p.plane_v = n_heads;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
+  p.out = out;
+  p.timeout_ns = 2000000000ull;
+  p.debug_skip_v_tile = -1;
+
+  CUtensorMap q_map, kv_map;
+  if (encode_q_map(&q_map, q, head_dim, n_heads, n_query) != 0) return WS_ERR_CUDA;
+  if (encode_kv_map(&kv_map, kv, head_dim, n_keys, (int64_t)2 * n_heads) != 0) return WS_ERR_CUDA;
+
+  if (cudaMemsetAsync(p.status, 0, sizeof(int), stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (launch_attention(q_map, kv_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
+  bool any_split = false;
+  for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
+    for (int h = 0; h < n_heads && !any_split; ++h) {
+      int c_first, pieces;
+      item_span(p.dec, qt, h, c_first, pieces);
+      any_split = pieces > 1;
+    }
+  if (any_split && launch_merge(p, head_dim, stream) != cudaSuccess) return WS_ERR_CUDA;
+  return WS_OK;
+}

@@ -16,6 +16,50 @@
 
 using namespace ws;
 
+// Work decomposition of one attention call (see Decomp in kernels.cuh).  The Q
+// tiles are grouped into lanes so that the lanes together hold one CTA per SM;
+// the group size minimises the iterations of the busiest CTA (ties: the
+// smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
+// iterations.  `forced` > 0 fixes the CTAs per lane.  Returns false when the
+// partial slots would not fit the workspace even with one CTA per lane.
+bool ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap) {
+  const int sms = sm_count();
+  d.n_qtiles = n_qtiles;
+  d.heads = heads;
+  d.tiles = tiles;
+  int best_g = 1, best_cpl = 1;
+  long long best_cost = -1;
+  int prev_lanes = -1;
+  for (int g = 1; g <= n_qtiles; ++g) {
+    const int lanes = (n_qtiles + g - 1) / g;
+    if (lanes == prev_lanes) continue;
+    prev_lanes = lanes;
+    const long long work = (long long)g * heads * tiles;
+    long long cpl = forced > 0 ? forced : std::max(1, sms / lanes);
+    cpl = std::min<long long>(cpl, std::max<long long>(1, forced > 0 ? work : work / 2));
+    cpl = std::min<long long>(cpl, kMaxLaneCtas);
+    const long long cost = (work + cpl - 1) / cpl;
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_g = g;
+      best_cpl = (int)cpl;
+    }
+  }
+  d.group = best_g;
+  d.lanes = (n_qtiles + best_g - 1) / best_g;
+  for (int cpl = best_cpl;; cpl = std::max(1, cpl / 2)) {
+    d.lane_ctas = cpl;
+    long long min_per = -1;
+    for (int ln = 0; ln < d.lanes; ++ln) {
+      const long long per = lane_per(d, ln);
+      if (min_per < 0 || per < min_per) min_per = per;
+    }
+    d.max_pieces = (int)((tiles + min_per - 1) / min_per) + 1;
+    if ((int64_t)n_qtiles * heads * d.max_pieces <= slot_cap) return true;
+    if (cpl == 1) return false;
+  }
+}
+
 struct EventPool {
   std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 end
   int used = 0;
@@ -123,50 +167,6 @@ int plan_runs(const ws_cache_config& cfg, const int64_t* slot_unit, const uint8_
   }
   *n_runs = n;
   return WS_OK;
-}
-
-// Work decomposition of one attention call (see Decomp in kernels.cuh).  The Q
-// tiles are grouped into lanes so that the lanes together hold one CTA per SM;
-// the group size minimises the iterations of the busiest CTA (ties: the
-// smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
-// iterations.  `forced` > 0 fixes the CTAs per lane.  Returns false when the
-// partial slots would not fit the workspace even with one CTA per lane.
-bool decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap) {
-  const int sms = sm_count();
-  d.n_qtiles = n_qtiles;
-  d.heads = heads;
-  d.tiles = tiles;
-  int best_g = 1, best_cpl = 1;
-  long long best_cost = -1;
-  int prev_lanes = -1;
-  for (int g = 1; g <= n_qtiles; ++g) {
-    const int lanes = (n_qtiles + g - 1) / g;
-    if (lanes == prev_lanes) continue;
-    prev_lanes = lanes;
-    const long long work = (long long)g * heads * tiles;
-    long long cpl = forced > 0 ? forced : std::max(1, sms / lanes);
-    cpl = std::min<long long>(cpl, std::max<long long>(1, forced > 0 ? work : work / 2));
-    cpl = std::min<long long>(cpl, kMaxLaneCtas);
-    const long long cost = (work + cpl - 1) / cpl;
-    if (best_cost < 0 || cost < best_cost) {
-      best_cost = cost;
-      best_g = g;
-      best_cpl = (int)cpl;
-    }
-  }
-  d.group = best_g;
-  d.lanes = (n_qtiles + best_g - 1) / best_g;
-  for (int cpl = best_cpl;; cpl = std::max(1, cpl / 2)) {
-    d.lane_ctas = cpl;
-    long long min_per = -1;
-    for (int ln = 0; ln < d.lanes; ++ln) {
-      const long long per = lane_per(d, ln);
-      if (min_per < 0 || per < min_per) min_per = per;
-    }
-    d.max_pieces = (int)((tiles + min_per - 1) / min_per) + 1;
-    if ((int64_t)n_qtiles * heads * d.max_pieces <= slot_cap) return true;
-    if (cpl == 1) return false;
-  }
 }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? WS_OK : WS_ERR_CUDA; }

@@ -81,6 +81,7 @@ def _declare(lib):
         "ws_profile_read": (C.c_int, [_P, C.POINTER(ws_profile)]),
         "ws_plan_visible": (C.c_int, [C.POINTER(ws_cache_config), C.POINTER(i64), C.POINTER(C.c_uint8), C.c_int,
                                       i64, C.POINTER(i32), C.POINTER(i32), i32, C.POINTER(i32)]),
+        "ws_attention_noalloc": (C.c_int, [_P, _P, _P, i32, i32, i32, i32, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -237,6 +238,12 @@ def ws_plan_visible(cfg: ws_cache_config, slot_unit, latent_ready, layer, unit, 
     nr = C.c_int32(0)
     st = lib().ws_plan_visible(C.byref(cfg), su, lr, layer, unit, rb, rw, max_runs, C.byref(nr))
     return st, [(rb[i], rw[i]) for i in range(nr.value)] if st == WS_OK else []
+
+
+def ws_attention_noalloc(q, kv, out, n_query, n_keys, n_heads, head_dim, stream=None, check=True):
+    """Attention over caller-owned K/V planes kv [2][H][Nk][D]; no device allocation."""
+    return _done(lib().ws_attention_noalloc(_ptr(q), _ptr(kv), _ptr(out), n_query, n_keys, n_heads, head_dim,
+                                            _stream(stream)), "ws_attention_noalloc", check)
 
 
 def synth_fill(dst, key: int, index0: int = 0, stream=None):

@@ -1,0 +1,78 @@
+"""ws_attention_noalloc -- attention for callers that cannot allocate device memory
+(graph captures without allocation nodes, frameworks that own every allocation,
+real-time loops) -- gives the same result as ws_unit_attention on the same keys,
+for two calls in a row that reuse its shared scratch array with different shapes.
+Kept in a file of its own, collected last."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import ATOL_MAX, ATOL_MEAN, require_gpu, to_dev
+from kv_cache_serving_ws_b200 import native as ws
+from kv_cache_serving_ws_b200 import synth
+
+
+def _reference_and_keys(cfg, layer, seed):
+    """Run ws_unit_attention on a small cache and return (q, out, kv planes [2][H][Nk][D])."""
+    L, H, D, Nv, Na, Nc, U = cfg
+    Nq = Nv + Na
+    _, h = ws.ws_cache_create(ws.make_config(L, H, D, Nv, Na, Nc, U))
+    bits = lambda kind, shape, u=0, l=0: to_dev(synth.normal_tensor(synth.stream_key(seed, kind, u, l), shape))
+    unit = U + 1
+    for u in range(unit + 1):
+        ws.ws_cache_append(h, u, ws.WS_SEG_COND, bits(synth.KIND_COND_K, (L, Nc, H, D), u),
+                           bits(synth.KIND_COND_V, (L, Nc, H, D), u))
+        if u < unit:
+            ws.ws_cache_append(h, u, ws.WS_SEG_LATENT, bits(synth.KIND_COMMIT_K, (L, Nq, H, D), u),
+                               bits(synth.KIND_COMMIT_V, (L, Nq, H, D), u))
+    q = bits(synth.KIND_Q, (Nq, H, D), unit, layer)
+    kn = bits(synth.KIND_K_NEW, (Nq, H, D), unit, layer)
+    vn = bits(synth.KIND_V_NEW, (Nq, H, D), unit, layer)
+    out = torch.empty_like(q)
+    ws.ws_unit_attention(h, layer, unit, q, kn, vn, out)
+    # the visible keys (units unit-U .. unit), read back from the cache
+    ks, vs = [], []
+    for u in range(unit - U, unit + 1):
+        for seg, n in ((ws.WS_SEG_COND, Nc), (ws.WS_SEG_LATENT, Nq)):
+            kb = torch.empty((n, H, D), dtype=torch.bfloat16, device="cuda")
+            vb = torch.empty_like(kb)
+            ws.ws_cache_read(h, layer, u, seg, kb, vb)
+            ks.append(kb)
+            vs.append(vb)
+    assert ws.ws_sync(h, check=False) == ws.WS_OK
+    ws.ws_cache_destroy(h)
+    k = torch.cat(ks).permute(1, 0, 2)          # [H][Nk][D]
+    v = torch.cat(vs).permute(1, 0, 2)
+    kv = torch.stack([k, v]).contiguous()       # [2][H][Nk][D]
+    return q, out, kv
+
+
+@pytest.mark.gpu
+def test_noalloc_matches_unit_attention_on_two_calls_in_a_row():
+    require_gpu()
+    cases = [((2, 6, 128, 250, 4, 16, 3), 1, 21),   # D = 128, key ranges cut between CTAs
+             ((1, 5, 64, 300, 7, 9, 2), 0, 22)]     # D = 64, other shapes: reuses the same scratch
+    for cfg, layer, seed in cases:
+        q, ref, kv = _reference_and_keys(cfg, layer, seed)
+        _, H, D, Nv, Na, _, _ = cfg
+        Nq, Nk = Nv + Na, kv.shape[2]
+        out = torch.full_like(q, float("nan"))
+        assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, check=False) == ws.WS_OK
+        torch.cuda.synchronize()
+        got = out.to(torch.float64).cpu().numpy()
+        want = ref.to(torch.float64).cpu().numpy()
+        assert np.all(np.isfinite(got))
+        d = np.abs(got - want)
+        assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (cfg, float(d.max()), float(d.mean()))
+
+
+@pytest.mark.gpu
+def test_noalloc_rejects_bad_arguments_before_any_launch():
+    require_gpu()
+    t = torch.zeros(64, dtype=torch.bfloat16, device="cuda")
+    assert ws.ws_attention_noalloc(t, t, t, 0, 8, 1, 64, check=False) == ws.WS_ERR_ARG
+    assert ws.ws_attention_noalloc(t, t, t, 1, 8, 1, 96, check=False) == ws.WS_ERR_UNSUPPORTED
+    odd = torch.zeros(80, dtype=torch.bfloat16, device="cuda")[1:65]
+    assert ws.ws_attention_noalloc(odd, t, t, 1, 1, 1, 64, check=False) == ws.WS_ERR_ALIGN
+    # partials of 4096 query tiles x 64 heads cannot fit the 48 MiB array
+    assert ws.ws_attention_noalloc(t, t, t, 4096 * 128, 1 << 20, 64, 128, check=False) == ws.WS_ERR_UNSUPPORTED
