@@ -78,47 +78,74 @@ struct Smem {
 __device__ __forceinline__ uint32_t tmem_s(uint32_t base, int b) { return base + (uint32_t)(b * 128); }
 __device__ __forceinline__ uint32_t tmem_o(uint32_t base) { return base + 256u; }
 
-__device__ __forceinline__ int tile_run(const KeyRuns& r, int t) {
-  int k = 0, hi = r.n_runs - 1;          // last run with tile_begin <= t
-  while (k < hi) {
-    const int mid = (k + hi + 1) >> 1;
-    if (r.tile_begin[mid] <= t) k = mid; else hi = mid - 1;
-  }
-  return k;
-}
-__device__ __forceinline__ int tile_row0(const KeyRuns& r, int t) {
-  const int k = tile_run(r, t);
-  return r.row_begin[k] + (t - r.tile_begin[k]) * kBlockN;
-}
-__device__ __forceinline__ int tile_valid(const KeyRuns& r, int t) {
-  const int k = tile_run(r, t);
-  return min(kBlockN, r.rows[k] - (t - r.tile_begin[k]) * kBlockN);
-}
-
-// Position of the CTA-local iteration g: Q tile, head, key tile, item ordinal
-// within the CTA, and whether g opens / closes its item.
-struct Iter {
-  int qt, h, t, n;
-  bool first, last;
-};
+// Walks a CTA's iterations in order: head h, Q tile qt, key tile t, item
+// ordinal n, and the key tile's run (first row, valid rows) -- all kept in
+// registers and advanced incrementally, so the hot loops do no divisions and
+// no indexed parameter loads except when a run or an item ends.
 struct Range {
   int lane, idx, gq;        // lane, CTA index in the lane, Q tiles of the lane
   long long start;          // first lane iteration
   int len;                  // iterations of this CTA
-  long long item0;          // lane-local item of the first iteration
 };
-__device__ __forceinline__ Iter iter_at(const Decomp& d, const Range& r, int g) {
-  const long long pos = r.start + g;
-  const long long item = pos / d.tiles;
-  Iter it;
-  it.t = (int)(pos - item * d.tiles);
-  it.h = (int)(item / r.gq);
-  it.qt = r.lane * d.group + (int)(item - (long long)it.h * r.gq);
-  it.n = (int)(item - r.item0);
-  it.first = (g == 0) || (it.t == 0);
-  it.last = (g == r.len - 1) || (it.t == d.tiles - 1);
-  return it;
-}
+struct TileIter {
+  int g, len, tiles, gq, qt0;
+  int t, a, h, n;
+  int run, run_off, run_row0, run_rows;
+  bool first, last;
+  __device__ __forceinline__ int qt() const { return qt0 + a; }
+  __device__ __forceinline__ int row0() const { return run_row0 + run_off; }
+  __device__ __forceinline__ int valid() const { return min(kBlockN, run_rows - run_off); }
+  __device__ __forceinline__ void flags() {
+    first = (g == 0) || (t == 0);
+    last = (g == len - 1) || (t == tiles - 1);
+  }
+  __device__ __forceinline__ void load_run(const KeyRuns& r) {
+    run_row0 = r.row_begin[run];
+    run_rows = r.rows[run];
+  }
+  __device__ void init(const Decomp& d, const KeyRuns& r, const Range& rg) {
+    g = 0;
+    len = rg.len;
+    tiles = d.tiles;
+    gq = rg.gq;
+    qt0 = rg.lane * d.group;
+    const long long item = rg.start / tiles;
+    t = (int)(rg.start - item * tiles);
+    h = (int)(item / gq);
+    a = (int)(item - (long long)h * gq);
+    n = 0;
+    run = 0;
+    int hi = r.n_runs - 1;                 // last run with tile_begin <= t
+    while (run < hi) {
+      const int mid = (run + hi + 1) >> 1;
+      if (r.tile_begin[mid] <= t) run = mid; else hi = mid - 1;
+    }
+    run_off = (t - r.tile_begin[run]) * kBlockN;
+    load_run(r);
+    flags();
+  }
+  __device__ __forceinline__ void next(const KeyRuns& r) {
+    ++g;
+    ++t;
+    run_off += kBlockN;
+    if (t == tiles) {
+      t = 0;
+      ++n;
+      if (++a == gq) {
+        a = 0;
+        ++h;
+      }
+      run = 0;
+      run_off = 0;
+      load_run(r);
+    } else if (run_off >= run_rows) {
+      ++run;
+      run_off = 0;
+      load_run(r);
+    }
+    flags();
+  }
+};
 
 // Bounded wait used only to drain in-flight copies and MMAs on the way out.
 __device__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
@@ -146,7 +173,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     rg.start = (long long)rg.idx * per;
     const long long end = rg.start + per < work ? rg.start + per : work;
     rg.len = end > rg.start ? (int)(end - rg.start) : 0;
-    rg.item0 = rg.start / d.tiles;
   }
   if (rg.len == 0) return;                 // whole CTA: nothing allocated yet
 
@@ -201,18 +227,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1}, last_q = -1;
       bool ok = true;
-      for (int g = 0; g < len && ok; ++g) {
-        const Iter it = iter_at(d, rg, g);
+      TileIter it;
+      it.init(d, p.runs, rg);
+      for (int g = 0; g < len && ok; ++g, it.next(p.runs)) {
         if (it.first) {
           if (it.n > 0 && !wait_phase(&bars[kQEmpty], (uint32_t)(it.n - 1) & 1, guard)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars[kQFull], S::kQTileBytes);
           for (int c = 0; c < S::kChunks; ++c)
-            tma_load_3d(sQ + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h, it.qt * kBlockM);
+            tma_load_3d(sQ + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h, it.qt() * kBlockM);
           last_q = it.n;
         }
         const int s = g & 1;
         const uint32_t use = (uint32_t)g >> 1;
-        const int row0 = tile_row0(p.runs, it.t);
+        const int row0 = it.row0();
         if (use > 0 && !wait_phase(&bars[kKEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars[kKFull + s], S::kTileBytes);
         for (int c = 0; c < S::kChunks; ++c)
@@ -244,8 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32(kBlockM, D, false, true);
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
       // S(g) = Q K(g)^T into S buffer g % 2
-      auto issue_s = [&](int g) -> bool {
-        const Iter it = iter_at(d, rg, g);
+      auto issue_s = [&](const TileIter& it) -> bool {
+        const int g = it.g;
         const int s = g & 1;
         if (it.first && !wait_phase(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
         if (!wait_phase(&bars[kKFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
@@ -265,8 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       // O += P(g) V(g), P(g) in the TMEM columns of S buffer g % 2
-      auto issue_pv = [&](int g) -> bool {
-        const Iter it = iter_at(d, rg, g);
+      auto issue_pv = [&](const TileIter& it) -> bool {
+        const int g = it.g;
         const int s = g & 1;
         if (!wait_phase(&bars[kVFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
         if (!wait_phase(&bars[kPFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
@@ -287,10 +314,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (it.last) umma_commit(&bars[kOFull]);
         return true;
       };
-      bool ok = issue_s(0);
+      TileIter it_s, it_pv;                  // it_s runs one iteration ahead of it_pv
+      it_s.init(d, p.runs, rg);
+      it_pv = it_s;
+      bool ok = issue_s(it_s);
       for (int g = 0; ok && g < len; ++g) {
-        if (g + 1 < len) ok = issue_s(g + 1);
-        if (ok) ok = issue_pv(g);
+        if (g + 1 < len) {
+          it_s.next(p.runs);
+          ok = issue_s(it_s);
+        }
+        if (ok) ok = issue_pv(it_pv);
+        it_pv.next(p.runs);
       }
       umma_commit(&bars[kMmaDone]);
       drain_wait(&bars[kMmaDone], 0, p.timeout_ns);
@@ -303,8 +337,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m_ref = -INFINITY;  // reference max of this row, log2 units
     float l_sum = 0.f;
     bool ok = true;
-    for (int g = 0; g < len; ++g) {
-      const Iter it = iter_at(d, rg, g);
+    TileIter it;
+    it.init(d, p.runs, rg);
+    for (int g = 0; g < len; ++g, it.next(p.runs)) {
       const int b = g & 1;
       const uint32_t t_s = tmem_s(tmem, b) + lane_base;
       if (it.first) {
@@ -316,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after_sync();
       uint32_t sr[kBlockN];
       tmem_load_128(t_s, sr);
-      const int valid = tile_valid(p.runs, it.t);
+      const int valid = it.valid();
       if (valid < kBlockN) {
 #pragma unroll
         for (int c = 0; c < kBlockN; ++c)
@@ -382,14 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_phase(&bars[kOFull], (uint32_t)it.n & 1, guard);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after_sync();
-        const int q_row = it.qt * kBlockM + row;
+        const int q_row = it.qt() * kBlockM + row;
         int c_first, pieces;
-        item_span(d, it.qt, it.h, c_first, pieces);
+        item_span(d, it.qt(), it.h, c_first, pieces);
         const float inv = 1.f / l_sum;
         uint16_t* dst = p.out + ((size_t)q_row * p.n_heads + it.h) * D;
         size_t prow = 0;
         if (pieces > 1) {
-          const size_t slot = ((size_t)it.qt * p.n_heads + it.h) * d.max_pieces + (size_t)(rg.idx - c_first);
+          const size_t slot = ((size_t)it.qt() * p.n_heads + it.h) * d.max_pieces + (size_t)(rg.idx - c_first);
           prow = slot * kBlockM + (size_t)row;
           *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
         }

@@ -6,8 +6,9 @@
 //
 // dt (an fp32) times a bf16 has at most 32 significant bits, so the fp64
 // product is exact; the sum is rounded once to fp64 and once to bf16 with
-// round-to-nearest-even.  The kernel moves 6 bytes per element and has ample
-// fp64 throughput for two fp64 operations per element at HBM speed.
+// round-to-nearest-even.  The kernel moves 6 bytes per element; per element it
+// spends one fp64 FMA and a few conversions, well within the fp64 rate at HBM
+// speed.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -18,72 +19,68 @@ namespace ws {
 
 namespace {
 
-// Round a double to the nearest bf16 (ties to even), from the IEEE 754 encoding:
-// keep the top 8 significant bits of the 53-bit significand (fewer below the
-// bf16 normal range, where the step is 2^-133), round the dropped bits half to
-// even, let a carry ripple into the exponent, saturate to infinity past the
-// largest finite value.  Every NaN becomes 0x7FC0.
-__device__ __forceinline__ uint32_t bf16_rne_from_f64(double d) {
-  const uint64_t b = static_cast<uint64_t>(__double_as_longlong(d));
-  const uint32_t sign = static_cast<uint32_t>(b >> 48) & 0x8000u;
-  const uint32_t bexp = static_cast<uint32_t>(b >> 52) & 0x7FFu;
-  const uint64_t frac = b & 0x000FFFFFFFFFFFFFull;
-  if (bexp == 0x7FFu) return frac ? 0x7FC0u : (sign | 0x7F80u);
-  if (bexp == 0u) return sign;                      // |d| < 2^-1022: far below half the smallest bf16 step
-  const int e = static_cast<int>(bexp) - 1023;      // |d| = 1.frac * 2^e
-  const uint64_t sig = frac | (1ull << 52);
-  int shift;
-  uint32_t bias;
-  if (e >= -126) {
-    shift = 45;                                     // 53 - 8 significant bits
-    bias = (static_cast<uint32_t>(e + 127) << 7) - 128u;
-  } else {
-    shift = -81 - e;                                // sig * 2^(e-52) / 2^-133
-    if (shift > 53) return sign;                    // below half the smallest subnormal step
-    bias = 0u;
-  }
-  uint64_t q = sig >> shift;
-  const uint64_t rem = sig & ((1ull << shift) - 1ull);
-  const uint64_t half = 1ull << (shift - 1);
-  if (rem > half || (rem == half && (q & 1ull))) ++q;
-  uint32_t mag = bias + static_cast<uint32_t>(q);
-  if (mag >= 0x7F80u) mag = 0x7F80u;
-  return sign | mag;
+// Round a double to the nearest bf16, ties to even, in two steps: to fp32 with
+// round-to-odd (truncate, then set the last bit when the truncation was
+// inexact), then fp32 -> bf16 with the hardware's round-to-nearest-even.
+// Rounding to odd at a precision with at least two more bits than the target
+// and then to nearest gives the correctly rounded result (Boldo and Melquiond,
+// "When double rounding is odd", 2005); fp32 keeps 16 more significant bits than
+// bf16 at every exponent, subnormals included.  Every NaN becomes 0x7FC0.
+__device__ __forceinline__ float f64_to_f32_odd(double d) {
+  const float t = __double2float_rz(d);
+  uint32_t u = __float_as_uint(t);
+  if (static_cast<double>(t) != d) u |= 1u;   // inexact (or NaN): sticky bit
+  return __uint_as_float(u);
 }
 
+__device__ __forceinline__ uint32_t bf16x2_rne_from_f64(double lo, double hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(f64_to_f32_odd(lo)), "f"(f64_to_f32_odd(hi)));
+  if (lo != lo) r = (r & 0xFFFF0000u) | 0x7FC0u;
+  if (hi != hi) r = (r & 0x0000FFFFu) | 0x7FC00000u;
+  return r;
+}
+
+// x + dt*v for two packed bf16 pairs: dt*v is exact in fp64, so one fused
+// multiply-add rounds the sum once, exactly as the separate product and sum do.
 __device__ __forceinline__ uint32_t euler2(uint32_t x2, uint32_t v2, double dt) {
   const double x_lo = static_cast<double>(__uint_as_float(x2 << 16));
   const double x_hi = static_cast<double>(__uint_as_float(x2 & 0xFFFF0000u));
   const double v_lo = static_cast<double>(__uint_as_float(v2 << 16));
   const double v_hi = static_cast<double>(__uint_as_float(v2 & 0xFFFF0000u));
-  const uint32_t lo = bf16_rne_from_f64(__dadd_rn(x_lo, __dmul_rn(dt, v_lo)));
-  const uint32_t hi = bf16_rne_from_f64(__dadd_rn(x_hi, __dmul_rn(dt, v_hi)));
-  return lo | (hi << 16);
+  return bf16x2_rne_from_f64(__fma_rn(dt, v_lo, x_lo), __fma_rn(dt, v_hi, x_hi));
 }
 
-__global__ void __launch_bounds__(256) euler_kernel(uint16_t* x, const uint16_t* v, float dt,
-                                                    int64_t n) {
+__device__ __forceinline__ uint4 euler8(uint4 a, const uint4 b, double dt) {
+  a.x = euler2(a.x, b.x, dt);
+  a.y = euler2(a.y, b.y, dt);
+  a.z = euler2(a.z, b.z, dt);
+  a.w = euler2(a.w, b.w, dt);
+  return a;
+}
+
+__global__ void __launch_bounds__(256) euler_kernel(uint16_t* x, const uint16_t* v, float dt, int64_t n) {
   const double dtd = static_cast<double>(dt);
   const int64_t nvec = n >> 3;
   uint4* xv = reinterpret_cast<uint4*>(x);
   const uint4* vv = reinterpret_cast<const uint4*>(v);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec; i += stride) {
-    uint4 a = xv[i];
-    const uint4 b = vv[i];
-    a.x = euler2(a.x, b.x, dtd);
-    a.y = euler2(a.y, b.y, dtd);
-    a.z = euler2(a.z, b.z, dtd);
-    a.w = euler2(a.w, b.w, dtd);
-    xv[i] = a;
+  int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  // two vectors per thread and iteration: four 16-byte loads in flight
+  for (; i + stride < nvec; i += 2 * stride) {
+    const uint4 a0 = xv[i], a1 = xv[i + stride];
+    const uint4 b0 = vv[i], b1 = vv[i + stride];
+    xv[i] = euler8(a0, b0, dtd);
+    xv[i + stride] = euler8(a1, b1, dtd);
   }
+  if (i < nvec) xv[i] = euler8(xv[i], vv[i], dtd);
   // ragged tail (n % 8 elements)
   if (blockIdx.x == 0) {
-    const int64_t i = (nvec << 3) + threadIdx.x;
-    if (threadIdx.x < 8 && i < n) {
-      const double xd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(x[i]) << 16));
-      const double vd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(v[i]) << 16));
-      x[i] = static_cast<uint16_t>(bf16_rne_from_f64(__dadd_rn(xd, __dmul_rn(dtd, vd))));
+    const int64_t j = (nvec << 3) + threadIdx.x;
+    if (threadIdx.x < 8 && j < n) {
+      const double xd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(x[j]) << 16));
+      const double vd = static_cast<double>(__uint_as_float(static_cast<uint32_t>(v[j]) << 16));
+      x[j] = static_cast<uint16_t>(bf16x2_rne_from_f64(__fma_rn(dtd, vd, xd), 0.0) & 0xFFFFu);
     }
   }
 }
