@@ -12,17 +12,19 @@
 // tile of each run masks the rows past its end.
 //
 // Persistent kernel, one CTA per SM, stream-K style: every CTA gets the same
-// number of (Q tile, head, key tile) iterations (see Decomp).  A CTA works on one
-// 128-row query tile of one head at a time:
-//   warps 0-3  softmax: one query row per thread (= one TMEM lane); fp32 online
-//              softmax in base 2 with a lazily moved reference max; P is rounded
-//              to bf16 and written back into the TMEM columns of its own S (A
-//              operand of the P.V product); epilogue of each item;
-//   warp 4     TMA producer: the Q tile of each item, K and V tiles (2 stages);
-//   warp 5     MMA issuer: S(j+1) = Q K(j+1)^T into the other of two TMEM S
-//              buffers before O += P(j) V(j) (A from TMEM, V as an MN-major B
-//              operand), so the next tile's QK^T overlaps this tile's softmax.
-// TMEM: S buffers [0,128) and [128,256), O [256, 256+D).
+// number of (Q block, head, key tile) iterations (see Decomp).  A CTA works on a
+// block of two 128-row query tiles of one head at a time:
+//   warpgroup 0, 1  softmax of query tile 0 and 1: one query row per thread (=
+//              one TMEM lane); fp32 online softmax in base 2 with a lazily moved
+//              reference max; P is rounded to bf16 and written back into the TMEM
+//              columns of its own S (A operand of the P.V product); epilogue of
+//              each item;
+//   warp 8     TMA producer: the two Q tiles of each item, K and V tiles (2 stages);
+//   warp 9     MMA issuer: S_a = Q_a K^T (A and B from shared memory) and
+//              O_a += P_a V (A from TMEM, V as an MN-major B operand), ordered
+//              PV0(j), S0(j+1), PV1(j), S1(j+1): while one warpgroup runs its
+//              softmax the tensor core works on the other tile's products.
+// TMEM: S0 [0,128), O0 [128,128+D), S1 [256,384), O1 [384,384+D).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -44,18 +46,19 @@ enum Bar : int {
   kKEmpty = 4,   // +stage
   kVFull = 6,    // +stage
   kVEmpty = 8,   // +stage
-  kSFull = 10,   // +S buffer
-  kPFull = 12,   // +S buffer
-  kPVDone = 14,
-  kOFull = 15,
-  kOFree = 16,
-  kMmaDone = 17,
-  kNumBars = 18
+  kSFull = 10,   // +Q tile
+  kPFull = 12,   // +Q tile
+  kOFull = 14,   // +Q tile
+  kOFree = 16,   // +Q tile
+  kMmaDone = 18,
+  kNumBars = 19
 };
 
-constexpr int kSoftmaxWarps = 4;
+constexpr int kSoftmaxWarps = 4 * kQTiles;
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;
+// 320 threads, one CTA per SM: three warps share some SM sub-partitions, which
+// caps a thread at 168 registers; the softmax fits without spills.
 constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
 constexpr int kTmemCols = 512;
 constexpr int kRowBytes = 128;   // one 128-byte swizzle row = 64 bf16
@@ -66,7 +69,7 @@ struct Smem {
   static constexpr int kQTileBytes = kBlockM * D * 2;
   static constexpr int kTileBytes = kBlockN * D * 2;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQTileBytes;
+  static constexpr int kOffK = kOffQ + kQTiles * kQTileBytes;
   static constexpr int kOffV = kOffK + 2 * kTileBytes;
   static constexpr int kOffBar = kOffV + 2 * kTileBytes;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -75,8 +78,8 @@ struct Smem {
   static constexpr int kAlloc = (kBytes + 1024) > 120 * 1024 ? (kBytes + 1024) : 120 * 1024;
 };
 
-__device__ __forceinline__ uint32_t tmem_s(uint32_t base, int b) { return base + (uint32_t)(b * 128); }
-__device__ __forceinline__ uint32_t tmem_o(uint32_t base) { return base + 256u; }
+__device__ __forceinline__ uint32_t tmem_s(uint32_t base, int a) { return base + (uint32_t)(a * 256); }
+__device__ __forceinline__ uint32_t tmem_o(uint32_t base, int a) { return base + (uint32_t)(a * 256 + 128); }
 
 // Walks a CTA's iterations in order: head h, Q tile qt, key tile t, item
 // ordinal n, and the key tile's run (first row, valid rows) -- all kept in
@@ -198,12 +201,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kKEmpty + s], 1);
       mbar_init(&bars[kVFull + s], 1);
       mbar_init(&bars[kVEmpty + s], 1);
-      mbar_init(&bars[kSFull + s], 1);
-      mbar_init(&bars[kPFull + s], 4);
     }
-    mbar_init(&bars[kPVDone], 1);
-    mbar_init(&bars[kOFull], 1);
-    mbar_init(&bars[kOFree], 4);
+    for (int a = 0; a < kQTiles; ++a) {
+      mbar_init(&bars[kSFull + a], 1);
+      mbar_init(&bars[kPFull + a], 4);
+      mbar_init(&bars[kOFull + a], 1);
+      mbar_init(&bars[kOFree + a], 4);
+    }
     mbar_init(&bars[kMmaDone], 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -222,9 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, p.status, p.timeout_ns};
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
+  if (warp >= kSoftmaxWarps) {
+    if (warp == kProducerWarp && lane == 0) {
+      // ---------------------------------------------------------- producer
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1}, last_q = -1;
       bool ok = true;
       TileIter it;
@@ -232,9 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int g = 0; g < len && ok; ++g, it.next(p.runs)) {
         if (it.first) {
           if (it.n > 0 && !wait_phase(&bars[kQEmpty], (uint32_t)(it.n - 1) & 1, guard)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[kQFull], S::kQTileBytes);
-          for (int c = 0; c < S::kChunks; ++c)
-            tma_load_3d(sQ + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h, it.qt() * kBlockM);
+          mbar_arrive_expect_tx(&bars[kQFull], kQTiles * S::kQTileBytes);
+          for (int a = 0; a < kQTiles; ++a)
+            for (int c = 0; c < S::kChunks; ++c)
+              tma_load_3d(sQ + a * S::kQTileBytes + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h,
+                          it.qt() * kItemRows + a * kBlockM);
           last_q = it.n;
         }
         const int s = g & 1;
@@ -263,67 +269,67 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_v[s] >= 0) drain_wait(&bars[kVFull + s], ((uint32_t)last_v[s] >> 1) & 1, p.timeout_ns);
         }
       }
-    }
-  } else if (warp == kMmaWarp) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    } else if (warp == kMmaWarp && lane == 0) {
+      // -------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32(kBlockM, D, false, true);
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
-      // S(g) = Q K(g)^T into S buffer g % 2
-      auto issue_s = [&](const TileIter& it) -> bool {
-        const int g = it.g;
-        const int s = g & 1;
-        if (it.first && !wait_phase(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
-        if (!wait_phase(&bars[kKFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
+      // S_a(g) = Q_a K(g)^T
+      auto issue_s = [&](const TileIter& it, int a) -> bool {
+        const int s = it.g & 1;
+        if (a == 0) {
+          if (it.first && !wait_phase(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
+          if (!wait_phase(&bars[kKFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+        }
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_s(tmem, s);
+        const uint32_t d_tmem = tmem_s(tmem, a);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (uint32_t)((kk >> 2) * kBlockM * kRowBytes + (kk & 3) * 32);
           const uint32_t koff = (uint32_t)((kk >> 2) * kBlockN * kRowBytes + (kk & 3) * 32);
-          const uint64_t da = umma_smem_desc_sw128(q_base + off, 16, 1024);
+          const uint64_t da = umma_smem_desc_sw128(q_base + a * S::kQTileBytes + off, 16, 1024);
           const uint64_t db = umma_smem_desc_sw128(k_base + s * S::kTileBytes + koff, 16, 1024);
           umma_bf16_ss(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[kSFull + s]);
-        umma_commit(&bars[kKEmpty + s]);
-        if (it.last) umma_commit(&bars[kQEmpty]);
+        umma_commit(&bars[kSFull + a]);
+        if (a == kQTiles - 1) {
+          umma_commit(&bars[kKEmpty + s]);
+          if (it.last) umma_commit(&bars[kQEmpty]);
+        }
         return true;
       };
-      // O += P(g) V(g), P(g) in the TMEM columns of S buffer g % 2
-      auto issue_pv = [&](const TileIter& it) -> bool {
-        const int g = it.g;
-        const int s = g & 1;
-        if (!wait_phase(&bars[kVFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
-        if (!wait_phase(&bars[kPFull + s], ((uint32_t)g >> 1) & 1, guard)) return false;
-        if (it.first && it.n > 0 && !wait_phase(&bars[kOFree], (uint32_t)(it.n - 1) & 1, guard)) return false;
+      // O_a += P_a(g) V(g), P_a in the TMEM columns of S_a, two bf16 per column
+      auto issue_pv = [&](const TileIter& it, int a) -> bool {
+        const int s = it.g & 1;
+        if (a == 0 && !wait_phase(&bars[kVFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+        if (!wait_phase(&bars[kPFull + a], (uint32_t)it.g & 1, guard)) return false;
+        if (it.first && it.n > 0 && !wait_phase(&bars[kOFree + a], (uint32_t)(it.n - 1) & 1, guard)) return false;
         tc_fence_after_sync();
-        const uint32_t o_tmem = tmem_o(tmem);
-        const uint32_t p_tmem = tmem_s(tmem, s);
+        const uint32_t o_tmem = tmem_o(tmem, a);
+        const uint32_t p_tmem = tmem_s(tmem, a);
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          // 16 keys = 8 TMEM columns of packed bf16 pairs; V: 16 rows of 128 bytes,
-          // the next 64 head-dim columns one chunk (kBlockN rows) further
+          // 16 keys = 8 TMEM columns; V: 16 rows of 128 bytes, the next 64
+          // head-dim columns one chunk (kBlockN rows) further
           const uint64_t db = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
                                                    kBlockN * kRowBytes, 1024);
           umma_bf16_ts(o_tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bars[kPVDone]);
-        umma_commit(&bars[kVEmpty + s]);
-        if (it.last) umma_commit(&bars[kOFull]);
+        if (it.last) umma_commit(&bars[kOFull + a]);
+        if (a == kQTiles - 1) umma_commit(&bars[kVEmpty + s]);
         return true;
       };
       TileIter it_s, it_pv;                  // it_s runs one iteration ahead of it_pv
       it_s.init(d, p.runs, rg);
       it_pv = it_s;
-      bool ok = issue_s(it_s);
+      bool ok = issue_s(it_s, 0) && issue_s(it_s, 1);
       for (int g = 0; ok && g < len; ++g) {
-        if (g + 1 < len) {
-          it_s.next(p.runs);
-          ok = issue_s(it_s);
-        }
-        if (ok) ok = issue_pv(it_pv);
+        const bool more = g + 1 < len;
+        if (more) it_s.next(p.runs);
+        ok = issue_pv(it_pv, 0);
+        if (ok && more) ok = issue_s(it_s, 0);
+        if (ok) ok = issue_pv(it_pv, 1);
+        if (ok && more) ok = issue_s(it_s, 1);
         it_pv.next(p.runs);
       }
       umma_commit(&bars[kMmaDone]);
@@ -331,22 +337,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------- softmax
-    const int row = threadIdx.x;             // TMEM lane
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_o = tmem_o(tmem) + lane_base;
+    const int a = warp >> 2;                 // query tile of this warpgroup
+    const int row = threadIdx.x & 127;       // TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t t_s = tmem_s(tmem, a) + lane_base;
+    const uint32_t t_o = tmem_o(tmem, a) + lane_base;
     float m_ref = -INFINITY;  // reference max of this row, log2 units
     float l_sum = 0.f;
     bool ok = true;
     TileIter it;
     it.init(d, p.runs, rg);
     for (int g = 0; g < len; ++g, it.next(p.runs)) {
-      const int b = g & 1;
-      const uint32_t t_s = tmem_s(tmem, b) + lane_base;
       if (it.first) {
         m_ref = -INFINITY;
         l_sum = 0.f;
       }
-      ok = wait_phase(&bars[kSFull + b], ((uint32_t)g >> 1) & 1, guard);
+      // S_a(g) complete; it was issued after P_a(g-1) V, which is complete too
+      ok = wait_phase(&bars[kSFull + a], (uint32_t)g & 1, guard);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after_sync();
       uint32_t sr[kBlockN];
@@ -391,14 +398,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       l_sum += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
-      tmem_store_64(t_s, pk);                // keys 2c, 2c+1 -> column c of the S buffer
-      if (g > 0) {
-        // O holds P(g-1) V(g-1) once this completes; needed before rescaling it
-        ok = wait_phase(&bars[kPVDone], (uint32_t)(g - 1) & 1, guard);
-        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-      }
+      tmem_store_64(t_s, pk);                // keys 2c, 2c+1 -> column c of S_a
       if (__any_sync(0xffffffffu, move && !it.first)) {
-        tc_fence_after_sync();
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
           uint32_t o[32];
@@ -410,14 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before_sync();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kPFull + b]);
+      if (lane == 0) mbar_arrive(&bars[kPFull + a]);
 
       if (it.last) {
-        // ---- epilogue of the item (qt, h)
-        ok = wait_phase(&bars[kOFull], (uint32_t)it.n & 1, guard);
+        // ---- epilogue of the item (qt, h), rows of query tile a
+        ok = wait_phase(&bars[kOFull + a], (uint32_t)it.n & 1, guard);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after_sync();
-        const int q_row = it.qt() * kBlockM + row;
+        const int q_row = it.qt() * kItemRows + a * kBlockM + row;
         int c_first, pieces;
         item_span(d, it.qt(), it.h, c_first, pieces);
         const float inv = 1.f / l_sum;
@@ -425,7 +426,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         size_t prow = 0;
         if (pieces > 1) {
           const size_t slot = ((size_t)it.qt() * p.n_heads + it.h) * d.max_pieces + (size_t)(rg.idx - c_first);
-          prow = slot * kBlockM + (size_t)row;
+          prow = slot * kItemRows + (size_t)(a * kBlockM + row);
           *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
         }
         // O in 32-column chunks: bf16 output of a whole item, fp32 partial otherwise
@@ -437,12 +438,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (q_row < p.n_query) {
 #pragma unroll
               for (int k = 0; k < 32; k += 8) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
-                w.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
-                w.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
-                w.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
-                *reinterpret_cast<uint4*>(dst + c + k) = w;
+                uint4 v;
+                v.x = pack_bf16x2(__uint_as_float(o[k + 0]) * inv, __uint_as_float(o[k + 1]) * inv);
+                v.y = pack_bf16x2(__uint_as_float(o[k + 2]) * inv, __uint_as_float(o[k + 3]) * inv);
+                v.z = pack_bf16x2(__uint_as_float(o[k + 4]) * inv, __uint_as_float(o[k + 5]) * inv);
+                v.w = pack_bf16x2(__uint_as_float(o[k + 6]) * inv, __uint_as_float(o[k + 7]) * inv);
+                *reinterpret_cast<uint4*>(dst + c + k) = v;
               }
             }
           } else {
@@ -454,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars[kOFree]);
+        if (lane == 0) mbar_arrive(&bars[kOFree + a]);
       }
     }
   }
@@ -478,20 +479,20 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Attn
   if (gw >= p.n_query * p.n_heads) return;
   const int row = gw / p.n_heads;
   const int h = gw - row * p.n_heads;
-  const int qt = row / kBlockM;
+  const int qt = row / kItemRows;
   int c_first, pieces;
   item_span(p.dec, qt, h, c_first, pieces);
   if (pieces == 1) return;                       // written directly by its CTA
   const size_t slot0 = ((size_t)qt * p.n_heads + h) * p.dec.max_pieces;
-  const int r = row - qt * kBlockM;
+  const int r = row - qt * kItemRows;
   float m_all = -INFINITY;
-  for (int k = 0; k < pieces; ++k) m_all = fmaxf(m_all, p.part_ml[((slot0 + k) * kBlockM + r) * 2]);
+  for (int k = 0; k < pieces; ++k) m_all = fmaxf(m_all, p.part_ml[((slot0 + k) * kItemRows + r) * 2]);
   float l_all = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   for (int k = 0; k < pieces; ++k) {
-    const size_t prow = (slot0 + k) * kBlockM + r;
+    const size_t prow = (slot0 + k) * kItemRows + r;
     const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
     const float w = ex2_approx(ml.x - m_all);
     l_all += w * ml.y;

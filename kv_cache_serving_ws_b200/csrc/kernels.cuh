@@ -7,6 +7,8 @@
 namespace ws {
 
 constexpr int kBlockM = 128;   // query rows per Q tile (one TMEM lane each)
+constexpr int kQTiles = 2;     // Q tiles per item (ping-pong softmax warpgroups)
+constexpr int kItemRows = kBlockM * kQTiles;
 constexpr int kBlockN = 128;   // keys per tile
 constexpr int kMaxRuns = 192;  // visible row runs per attention call (>= slots of any ring with gaps)
 constexpr int kMaxLaneCtas = 1024;
@@ -21,17 +23,18 @@ struct KeyRuns {
   int32_t tile_begin[kMaxRuns + 1];
 };
 
-// Work decomposition.  An item is (Q tile qt, head h) over all key tiles.  The
-// Q tiles are cut into lanes of `group` consecutive tiles; every lane has
-// `lane_ctas` CTAs, and CTA idx of a lane processes the iterations
-// [idx*per, (idx+1)*per) of its lane's (head, Q tile of the lane, key tile)
-// sequence, head major.  CTAs with the same idx in different lanes then read
-// the same K/V tiles at about the same time (L2 reuse).  An item covered by
-// one CTA is written as bf16 directly; an item cut between CTAs is written as
-// fp32 partials (slot item*max_pieces + piece, item = qt*H + h) and merged.
+// Work decomposition.  An item is (Q block qt of kItemRows rows, head h) over
+// all key tiles.  The Q blocks are cut into lanes of `group` consecutive
+// blocks; every lane has `lane_ctas` CTAs, and CTA idx of a lane processes the
+// iterations [idx*per, (idx+1)*per) of its lane's (head, Q block of the lane,
+// key tile) sequence, head major.  CTAs with the same idx in different lanes
+// then read the same K/V tiles at about the same time (L2 reuse).  An item
+// covered by one CTA is written as bf16 directly; an item cut between CTAs is
+// written as fp32 partials (slot item*max_pieces + piece, item = qt*H + h) and
+// merged.
 struct Decomp {
-  int32_t n_qtiles;
-  int32_t group;            // Q tiles per lane
+  int32_t n_qtiles;         // Q blocks of kItemRows rows
+  int32_t group;            // Q blocks per lane
   int32_t lanes;
   int32_t lane_ctas;
   int32_t tiles;            // key tiles per item
@@ -66,8 +69,8 @@ struct AttnParams {
   int32_t plane_v;          // same for V
   float scale_log2;         // log2(e) / sqrt(D)
   uint16_t* out;            // [Nq][H][D] bf16
-  float* part_o;            // [n_qtiles*H*max_pieces][kBlockM][D] fp32
-  float* part_ml;           // [n_qtiles*H*max_pieces][kBlockM][2] (reference max in log2 units, sum)
+  float* part_o;            // [n_qtiles*H*max_pieces][kItemRows][D] fp32
+  float* part_ml;           // [n_qtiles*H*max_pieces][kItemRows][2] (reference max in log2 units, sum)
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
   int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)

@@ -76,8 +76,8 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   p.runs.total_tiles = p.runs.tile_begin[1];
 
   // scratch layout: [status | part_ml | part_o]; slots sized for this call
-  const int n_qtiles = (n_query + kBlockM - 1) / kBlockM;
-  const size_t slot_bytes = (size_t)kBlockM * (head_dim + 2) * sizeof(float);
+  const int n_qtiles = (n_query + kItemRows - 1) / kItemRows;
+  const size_t slot_bytes = (size_t)kItemRows * (head_dim + 2) * sizeof(float);
   const int64_t slot_cap = (int64_t)((kScratchBytes - kStatusBytes) / slot_bytes);
   if (!decompose(p.dec, n_qtiles, n_heads, p.runs.total_tiles, 0, slot_cap)) return WS_ERR_UNSUPPORTED;
   const size_t slots = (size_t)n_qtiles * n_heads * p.dec.max_pieces;
@@ -88,7 +88,7 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   unsigned char* b = static_cast<unsigned char*>(base);
   p.status = reinterpret_cast<int*>(b);
   p.part_ml = reinterpret_cast<float*>(b + kStatusBytes);
-  p.part_o = reinterpret_cast<float*>(b + kStatusBytes + slots * kBlockM * 2 * sizeof(float));
+  p.part_o = reinterpret_cast<float*>(b + kStatusBytes + slots * kItemRows * 2 * sizeof(float));
 
   p.n_query = n_query;
   p.n_heads = n_heads;

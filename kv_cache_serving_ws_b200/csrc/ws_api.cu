@@ -229,10 +229,10 @@ int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t s
   const int64_t rows = (int64_t)h->C * h->T;
   h->kv_bytes = (size_t)L * 2 * H * rows * D * 2;
   // partial slots: items x (ceil(SMs / H) + 1) bounds every automatic decomposition
-  const int64_t n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
+  const int64_t n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
   h->slot_cap = n_qtiles * H * ((sm_count() + H - 1) / H + 1);
-  const size_t part_o_bytes = (size_t)h->slot_cap * kBlockM * D * 4;
-  const size_t part_ml_bytes = (size_t)h->slot_cap * kBlockM * 2 * 4;
+  const size_t part_o_bytes = (size_t)h->slot_cap * kItemRows * D * 4;
+  const size_t part_ml_bytes = (size_t)h->slot_cap * kItemRows * 2 * 4;
   h->ws_bytes = part_o_bytes + part_ml_bytes;
   int st = WS_OK;
   if (cudaMalloc(&h->kv, h->kv_bytes) != cudaSuccess || cudaMalloc(&h->part_o, part_o_bytes) != cudaSuccess ||
@@ -359,7 +359,7 @@ int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q,
   // 2. attention (+ merge of split partials)
   p.n_query = h->Nq;
   p.n_heads = H;
-  const int n_qtiles = (h->Nq + kBlockM - 1) / kBlockM;
+  const int n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
   if (!decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas, h->slot_cap)) return WS_ERR_UNSUPPORTED;
   bool any_split = false;
   for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
