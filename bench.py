@@ -500,6 +500,8 @@ def run_case(args):
     g.prefill()
     q, kn, vn = g.step_inputs(0)
     out = torch.empty_like(q)
+    for _ in range(2):                       # warm-up: first-call set-up, caches
+        ws.ws_unit_attention(g.h, 0, w.unit, q, kn, vn, out)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record()

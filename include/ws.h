@@ -200,7 +200,7 @@ const char* ws_status_string(int status);
 /*
  * Launch accounting of the attention path, for benchmarks.  While enabled, the
  * library records a CUDA event pair around each attention kernel and each
- * combine kernel it launches (on the caller's stream).  ws_profile_read
+ * merge kernel (combine_*) it launches (on the caller's stream).  ws_profile_read
  * synchronises those events and returns the totals since the last reset.
  */
 typedef struct {
