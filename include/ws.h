@@ -219,6 +219,17 @@ int ws_profile_enable(ws_cache_t* h, int enable);   /* enabling resets the total
 int ws_profile_read(ws_cache_t* h, ws_profile* out);
 
 /*
+ * ws_debug_inject_stall -- test hook for the failure-detection path.  While
+ * tile >= 0, every attention kernel of this cache leaves out the V load of its
+ * CTA-local key tile `tile`, so each CTA's bounded wait for it runs out: the
+ * kernel leaves its loops, drains its copies, frees TMEM and stores
+ * WS_ERR_DEVICE_TIMEOUT for ws_sync (the output of that call is undefined).
+ * tile = -1 turns it off.  The wait bound is 2 s, or WS_WAIT_TIMEOUT_MS (read
+ * when the cache is created).
+ */
+int ws_debug_inject_stall(ws_cache_t* h, int tile);
+
+/*
  * ws_plan_visible -- host-only planning step of ws_unit_attention, exposed for
  * tests: the key rows of one (layer, head) plane that a query of `unit` sees,
  * as maximal runs of consecutive rows [row_begin[i], row_begin[i] + rows[i]).

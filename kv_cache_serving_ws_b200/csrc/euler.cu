@@ -66,14 +66,17 @@ __global__ void __launch_bounds__(256) euler_kernel(uint16_t* x, const uint16_t*
   const uint4* vv = reinterpret_cast<const uint4*>(v);
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  // two vectors per thread and iteration: four 16-byte loads in flight
-  for (; i + stride < nvec; i += 2 * stride) {
-    const uint4 a0 = xv[i], a1 = xv[i + stride];
-    const uint4 b0 = vv[i], b1 = vv[i + stride];
-    xv[i] = euler8(a0, b0, dtd);
-    xv[i + stride] = euler8(a1, b1, dtd);
+  // four vectors per thread and iteration: eight 16-byte loads in flight
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    uint4 a[4], b[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) a[k] = xv[i + k * stride];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) b[k] = vv[i + k * stride];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) xv[i + k * stride] = euler8(a[k], b[k], dtd);
   }
-  if (i < nvec) xv[i] = euler8(xv[i], vv[i], dtd);
+  for (; i < nvec; i += stride) xv[i] = euler8(xv[i], vv[i], dtd);
   // ragged tail (n % 8 elements)
   if (blockIdx.x == 0) {
     const int64_t j = (nvec << 3) + threadIdx.x;

@@ -451,6 +451,12 @@ int ws_cache_set_splits(ws_cache_t* h, int n_split) {
   return WS_OK;
 }
 
+int ws_debug_inject_stall(ws_cache_t* h, int tile) {
+  if (!h || tile < -1) return WS_ERR_ARG;
+  h->debug_skip_v_tile = tile;
+  return WS_OK;
+}
+
 int ws_sync(ws_cache_t* h, cudaStream_t stream) {
   if (!h) return WS_ERR_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return WS_ERR_CUDA;

@@ -82,6 +82,7 @@ def _declare(lib):
         "ws_plan_visible": (C.c_int, [C.POINTER(ws_cache_config), C.POINTER(i64), C.POINTER(C.c_uint8), C.c_int,
                                       i64, C.POINTER(i32), C.POINTER(i32), i32, C.POINTER(i32)]),
         "ws_attention_noalloc": (C.c_int, [_P, _P, _P, i32, i32, i32, i32, _P]),
+        "ws_debug_inject_stall": (C.c_int, [_P, C.c_int]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -216,6 +217,11 @@ def ws_cache_set_splits(h, n_split, check=True):
 
 def ws_sync(h, stream=None, check=True):
     return _done(lib().ws_sync(h, _stream(stream)), "ws_sync", check)
+
+
+def ws_debug_inject_stall(h, tile, check=True):
+    """Test hook: leave out one V load per CTA so the kernel's bounded wait runs out (-1 = off)."""
+    return _done(lib().ws_debug_inject_stall(h, tile), "ws_debug_inject_stall", check)
 
 
 def ws_profile_enable(h, enable=True, check=True):
