@@ -364,16 +364,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int c = 0; c < kBlockN; ++c)
           if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
       }
+      // row max: 8 independent chains of three-input max
       float mx[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
 #pragma unroll
-      for (int c = 8; c < kBlockN; c += 8)
+      for (int c = 8; c < kBlockN; c += 16)
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], __uint_as_float(sr[c + k]));
+        for (int k = 0; k < 8; ++k) mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
       const float m_cand =
-          fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) *
-          p.scale_log2;
+          max3_f32(max3_f32(mx[0], mx[1], mx[2]), max3_f32(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.scale_log2;
       // Move the reference max only when P would exceed 2^8 (or for a new item).
       const bool move = it.first || m_cand > m_ref + 8.f;
       float alpha = 1.f;
@@ -382,21 +382,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         l_sum *= alpha;
         m_ref = m_cand;
       }
-      const float neg_m = -m_ref;
-      float rs[8];
+      // P = 2^(s * log2(e)/sqrt(D) - m): scale and shift on fp32 pairs, one ex2
+      // per element, sums on fp32 pairs (4 independent chains)
+      const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2);
+      const uint64_t negm2 = f32x2(-m_ref, -m_ref);
+      uint64_t rs2[4];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) rs[k] = 0.f;
+      for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
       uint32_t pk[kBlockN / 2];
 #pragma unroll
-      for (int c = 0; c < kBlockN; c += 16) {
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float e0 = ex2_approx(fmaf(__uint_as_float(sr[c + 2 * k]), p.scale_log2, neg_m));
-          const float e1 = ex2_approx(fmaf(__uint_as_float(sr[c + 2 * k + 1]), p.scale_log2, neg_m));
-          rs[k] += e0 + e1;
-          pk[c / 2 + k] = pack_bf16x2(e0, e1);
-        }
+      for (int c = 0; c < kBlockN / 2; ++c) {
+        const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
+        float x0, x1;
+        f32x2_split(x, x0, x1);
+        const float e0 = ex2_approx(x0);
+        const float e1 = ex2_approx(x1);
+        rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
+        pk[c] = pack_bf16x2(e0, e1);
       }
+      float rs[8];
+      f32x2_split(rs2[0], rs[0], rs[1]);
+      f32x2_split(rs2[1], rs[2], rs[3]);
+      f32x2_split(rs2[2], rs[4], rs[5]);
+      f32x2_split(rs2[3], rs[6], rs[7]);
       l_sum += ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
       tmem_store_64(t_s, pk);                // keys 2c, 2c+1 -> column c of S_a
       if (__any_sync(0xffffffffu, move && !it.first)) {
