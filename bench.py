@@ -517,6 +517,56 @@ def run_case(args):
         sys.exit(1)
 
 
+def run_prefill(args):
+    """Prompt prefill: n query units of the 640x368 stream attend at once, each over its
+    own window (block-causal across units), one layer; reports TFLOP/s of the useful
+    work and the key tiles the block-causal mask skips compared with a dense one."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200 import synth
+    from kv_cache_serving_ws_b200.workloads import Workload, key
+    n = args.prefill_units
+    w = Workload("prefill-640x368-40x128", 1, 40, 128, 920, 4, 32, 64, seed=6, unit=0)
+    _, h = ws.ws_cache_create(ws.make_config(1, w.n_heads, w.head_dim, w.n_video, w.n_audio, w.n_cond,
+                                             w.history_units))
+    dev = torch.device("cuda")
+    ck = torch.empty((1, w.n_cond, w.n_heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+    cv = torch.empty_like(ck)
+    for u in range(n):
+        ws.synth_fill(ck, key(w, synth.KIND_COND_K, u))
+        ws.synth_fill(cv, key(w, synth.KIND_COND_V, u))
+        ws.ws_cache_append(h, u, ws.WS_SEG_COND, ck, cv)
+    shape = (n, w.n_query, w.n_heads, w.head_dim)
+    q = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    kn, vn, out = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws.synth_fill(q, key(w, synth.KIND_Q, 0))
+    ws.synth_fill(kn, key(w, synth.KIND_K_NEW, 0))
+    ws.synth_fill(vn, key(w, synth.KIND_V_NEW, 0))
+    for _ in range(2):
+        ws.ws_prefill_attention(h, 0, 0, n, q, kn, vn, out)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.calls):
+        ws.ws_prefill_attention(h, 0, 0, n, q, kn, vn, out)
+    e1.record()
+    st = ws.ws_sync(h, check=False)
+    ms = e0.elapsed_time(e1) / args.calls
+    T = w.tokens_per_unit
+    keys = [min(j, w.history_units) * T + T for j in range(n)]           # window of query unit j (from scratch)
+    flops = sum(4.0 * w.n_query * k * w.n_heads * w.head_dim for k in keys)
+    tiles = sum((k + 127) // 128 for k in keys)
+    dense_tiles = n * ((n * T + 127) // 128)
+    print(json.dumps({"mode": "prefill", "workload": w.name, "query_units": n, "query_rows": n * w.n_query,
+                      "ms_per_call": round(ms, 3), "TFLOP/s": round(flops / ms / 1e9, 1),
+                      "key_tiles": tiles, "dense_mask_key_tiles": dense_tiles,
+                      "skipped_tile_fraction": round(1 - tiles / dense_tiles, 4), "status": ws.status_string(st)}))
+    ws.ws_cache_destroy(h)
+    if st != ws.WS_OK:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -528,9 +578,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--case", default=None, help="profiling mode: tiny|v01|v02|ring (attention calls only)")
     ap.add_argument("--calls", type=int, default=3)
+    ap.add_argument("--prefill", action="store_true", help="time a multi-unit prompt prefill instead")
+    ap.add_argument("--prefill-units", type=int, default=64)
     args = ap.parse_args()
     if args.case:
         run_case(args)
+        return
+    if args.prefill:
+        run_prefill(args)
         return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

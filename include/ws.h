@@ -141,6 +141,27 @@ int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit,
                       uint16_t* out, cudaStream_t stream);
 
 /*
+ * ws_prefill_attention -- block-causal attention of several consecutive query
+ * units at once (a prompt prefill or any full recomputation of a stretch of
+ * units), in one launch.  Query unit j = unit_first + j uses rows
+ * [j*Nq, (j+1)*Nq) of q, k_new, v_new and out ([n_units][Nq][H][D]); like
+ * ws_unit_attention it first writes each unit's k_new, v_new into its latent
+ * rows of `layer`, then every row of unit j sees the tokens of the resident
+ * units j - U .. j, never those of a later unit (block-causal across units,
+ * remio.ai, section 为什么端到端模型对级联式 AI 智能体构成挑战).  Key tiles of
+ * units outside a query unit's window are never loaded.  All query units must
+ * have their conditioning slice appended, the last one being the newest unit;
+ * 1 <= n_units <= 64.
+ * Errors: as ws_unit_attention; WS_ERR_NOT_READY / WS_ERR_EVICTED if a query
+ * unit is not resident; WS_ERR_EVICTED if a unit inside some query window has
+ * been overwritten (n_units larger than the ring allows); WS_ERR_UNSUPPORTED
+ * for n_units > 64.
+ */
+int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n_units,
+                         const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new,
+                         uint16_t* out, cudaStream_t stream);
+
+/*
  * ws_flow_step -- fused flow-matching Euler update, in place:
  *     x[i] <- RN_bf16( fl64( x[i] + fl64(dt * v[i]) ) ),   0 <= i < n
  * (paper.rainbus.top, section 核心方法).  dt*v is exact in fp64; the sum is

@@ -81,18 +81,18 @@ struct Smem {
 __device__ __forceinline__ uint32_t tmem_s(uint32_t base, int a) { return base + (uint32_t)(a * 256); }
 __device__ __forceinline__ uint32_t tmem_o(uint32_t base, int a) { return base + (uint32_t)(a * 256 + 128); }
 
-// Walks a CTA's iterations in order: head h, Q tile qt, key tile t, item
-// ordinal n, and the key tile's run (first row, valid rows) -- all kept in
-// registers and advanced incrementally, so the hot loops do no divisions and
-// no indexed parameter loads except when a run or an item ends.
+// Walks a CTA's iterations in order: head h, query block of the lane a, query
+// unit j, key tile t, item ordinal n, and the key tile's run (first row, valid
+// rows) -- all kept in registers and advanced incrementally, so the hot loops do
+// no divisions and no indexed parameter loads except when a run or an item ends.
 struct Range {
-  int lane, idx, gq;        // lane, CTA index in the lane, Q tiles of the lane
+  int lane, idx, gq;        // lane, CTA index in the lane, query blocks of the lane
   long long start;          // first lane iteration
   int len;                  // iterations of this CTA
 };
 struct TileIter {
-  int g, len, tiles, gq, qt0;
-  int t, a, h, n;
+  int g, len, tiles, gq, qt0, n_units;
+  int a, h, j, t, tiles_j, n;
   int run, run_off, run_row0, run_rows;
   bool first, last;
   __device__ __forceinline__ int qt() const { return qt0 + a; }
@@ -100,45 +100,50 @@ struct TileIter {
   __device__ __forceinline__ int valid() const { return min(kBlockN, run_rows - run_off); }
   __device__ __forceinline__ void flags() {
     first = (g == 0) || (t == 0);
-    last = (g == len - 1) || (t == tiles - 1);
+    last = (g == len - 1) || (t == tiles_j - 1);
   }
   __device__ __forceinline__ void load_run(const KeyRuns& r) {
     run_row0 = r.row_begin[run];
     run_rows = r.rows[run];
   }
-  __device__ void init(const Decomp& d, const KeyRuns& r, const Range& rg) {
+  __device__ void init(const Decomp& d, const QueryUnits& u, const KeyRuns& r, const Range& rg) {
     g = 0;
     len = rg.len;
     tiles = d.tiles;
     gq = rg.gq;
     qt0 = rg.lane * d.group;
-    const long long item = rg.start / tiles;
-    t = (int)(rg.start - item * tiles);
-    h = (int)(item / gq);
-    a = (int)(item - (long long)h * gq);
+    n_units = u.n_units;
+    const long long grp = rg.start / tiles;
+    const int rem = (int)(rg.start - grp * tiles);
+    h = (int)(grp / gq);
+    a = (int)(grp - (long long)h * gq);
+    j = 0;
+    while (j + 1 < n_units && u.tile_start[j + 1] <= rem) ++j;
+    t = rem - u.tile_start[j];
+    tiles_j = u.tile_start[j + 1] - u.tile_start[j];
     n = 0;
-    run = 0;
-    int hi = r.n_runs - 1;                 // last run with tile_begin <= t
-    while (run < hi) {
-      const int mid = (run + hi + 1) >> 1;
-      if (r.tile_begin[mid] <= t) run = mid; else hi = mid - 1;
-    }
+    run = u.run_first[j];
+    while (run + 1 < u.run_first[j + 1] && r.tile_begin[run + 1] <= t) ++run;
     run_off = (t - r.tile_begin[run]) * kBlockN;
     load_run(r);
     flags();
   }
-  __device__ __forceinline__ void next(const KeyRuns& r) {
+  __device__ __forceinline__ void next(const QueryUnits& u, const KeyRuns& r) {
     ++g;
     ++t;
     run_off += kBlockN;
-    if (t == tiles) {
+    if (t == tiles_j) {
       t = 0;
       ++n;
-      if (++a == gq) {
-        a = 0;
-        ++h;
+      if (++j == n_units) {
+        j = 0;
+        if (++a == gq) {
+          a = 0;
+          ++h;
+        }
       }
-      run = 0;
+      tiles_j = u.tile_start[j + 1] - u.tile_start[j];
+      run = u.run_first[j];
       run_off = 0;
       load_run(r);
     } else if (run_off >= run_rows) {
@@ -232,15 +237,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       int last_k[2] = {-1, -1}, last_v[2] = {-1, -1}, last_q = -1;
       bool ok = true;
       TileIter it;
-      it.init(d, p.runs, rg);
-      for (int g = 0; g < len && ok; ++g, it.next(p.runs)) {
+      it.init(d, p.qu, p.runs, rg);
+      for (int g = 0; g < len && ok; ++g, it.next(p.qu, p.runs)) {
         if (it.first) {
           if (it.n > 0 && !wait_phase(&bars[kQEmpty], (uint32_t)(it.n - 1) & 1, guard)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars[kQFull], kQTiles * S::kQTileBytes);
           for (int a = 0; a < kQTiles; ++a)
             for (int c = 0; c < S::kChunks; ++c)
               tma_load_3d(sQ + a * S::kQTileBytes + c * kBlockM * kRowBytes, &q_map, &bars[kQFull], c * 64, it.h,
-                          it.qt() * kItemRows + a * kBlockM);
+                          it.j * p.qu.rows + it.qt() * kItemRows + a * kBlockM);
           last_q = it.n;
         }
         const int s = g & 1;
@@ -320,17 +325,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         return true;
       };
       TileIter it_s, it_pv;                  // it_s runs one iteration ahead of it_pv
-      it_s.init(d, p.runs, rg);
+      it_s.init(d, p.qu, p.runs, rg);
       it_pv = it_s;
       bool ok = issue_s(it_s, 0) && issue_s(it_s, 1);
       for (int g = 0; ok && g < len; ++g) {
         const bool more = g + 1 < len;
-        if (more) it_s.next(p.runs);
+        if (more) it_s.next(p.qu, p.runs);
         ok = issue_pv(it_pv, 0);
         if (ok && more) ok = issue_s(it_s, 0);
         if (ok) ok = issue_pv(it_pv, 1);
         if (ok && more) ok = issue_s(it_s, 1);
-        it_pv.next(p.runs);
+        it_pv.next(p.qu, p.runs);
       }
       umma_commit(&bars[kMmaDone]);
       drain_wait(&bars[kMmaDone], 0, p.timeout_ns);
@@ -346,8 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float l_sum = 0.f;
     bool ok = true;
     TileIter it;
-    it.init(d, p.runs, rg);
-    for (int g = 0; g < len; ++g, it.next(p.runs)) {
+    it.init(d, p.qu, p.runs, rg);
+    for (int g = 0; g < len; ++g, it.next(p.qu, p.runs)) {
       if (it.first) {
         m_ref = -INFINITY;
         l_sum = 0.f;
@@ -426,14 +431,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_phase(&bars[kOFull + a], (uint32_t)it.n & 1, guard);
         if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
         tc_fence_after_sync();
-        const int q_row = it.qt() * kItemRows + a * kBlockM + row;
-        int c_first, pieces;
-        item_span(d, it.qt(), it.h, c_first, pieces);
+        const int r_unit = it.qt() * kItemRows + a * kBlockM + row;   // row within the query unit
+        int lane_i, c_first, pieces, end0;
+        item_span(d, p.qu, it.j, it.qt(), it.h, lane_i, c_first, pieces, end0);
         const float inv = 1.f / l_sum;
-        uint16_t* dst = p.out + ((size_t)q_row * p.n_heads + it.h) * D;
+        const bool in_unit = r_unit < p.qu.rows;
+        uint16_t* dst = p.out + ((size_t)(it.j * p.qu.rows + r_unit) * p.n_heads + it.h) * D;
         size_t prow = 0;
         if (pieces > 1) {
-          const size_t slot = ((size_t)it.qt() * p.n_heads + it.h) * d.max_pieces + (size_t)(rg.idx - c_first);
+          // this CTA's first item takes slot (cta, 0), any later one slot (cta, 1)
+          const size_t slot = partial_slot(d, rg.lane, rg.idx, it.n == 0 ? 0 : 1);
           prow = slot * kItemRows + (size_t)(a * kBlockM + row);
           *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
         }
@@ -443,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t o[32];
           tmem_load_32(t_o + (uint32_t)c, o);
           if (pieces == 1) {
-            if (q_row < p.n_query) {
+            if (in_unit) {
 #pragma unroll
               for (int k = 0; k < 32; k += 8) {
                 uint4 v;
@@ -484,23 +491,31 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Attn
   constexpr int kPer = D / 32;
   const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
-  if (gw >= p.n_query * p.n_heads) return;
+  const int rows = p.qu.n_units * p.qu.rows;
+  if (gw >= rows * p.n_heads) return;
   const int row = gw / p.n_heads;
   const int h = gw - row * p.n_heads;
-  const int qt = row / kItemRows;
-  int c_first, pieces;
-  item_span(p.dec, qt, h, c_first, pieces);
+  const int j = row / p.qu.rows;
+  const int r_unit = row - j * p.qu.rows;
+  const int qt = r_unit / kItemRows;
+  const int r = r_unit - qt * kItemRows;
+  int lane_i, c_first, pieces, end0;
+  item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
   if (pieces == 1) return;                       // written directly by its CTA
-  const size_t slot0 = ((size_t)qt * p.n_heads + h) * p.dec.max_pieces;
-  const int r = row - qt * kItemRows;
+  // piece k was written by CTA c_first + k: its last item for k = 0 (unless
+  // the item starts exactly at that CTA's range), its first item otherwise
   float m_all = -INFINITY;
-  for (int k = 0; k < pieces; ++k) m_all = fmaxf(m_all, p.part_ml[((slot0 + k) * kItemRows + r) * 2]);
+  for (int k = 0; k < pieces; ++k) {
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    m_all = fmaxf(m_all, p.part_ml[(slot * kItemRows + r) * 2]);
+  }
   float l_all = 0.f;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
   for (int k = 0; k < pieces; ++k) {
-    const size_t prow = (slot0 + k) * kItemRows + r;
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    const size_t prow = slot * kItemRows + r;
     const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
     const float w = ex2_approx(ml.x - m_all);
     l_all += w * ml.y;
@@ -598,7 +613,7 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
 }
 
 cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  const long long warps = (long long)p.n_query * p.n_heads;
+  const long long warps = (long long)p.qu.n_units * p.qu.rows * p.n_heads;
   const int grid = (int)((warps * 32 + 255) / 256);
   if (head_dim == 128)
     merge_kernel<128><<<grid, 256, 0, stream>>>(p);

@@ -10,36 +10,48 @@ constexpr int kBlockM = 128;   // query rows per Q tile (one TMEM lane each)
 constexpr int kQTiles = 2;     // Q tiles per item (ping-pong softmax warpgroups)
 constexpr int kItemRows = kBlockM * kQTiles;
 constexpr int kBlockN = 128;   // keys per tile
-constexpr int kMaxRuns = 192;  // visible row runs per attention call (>= slots of any ring with gaps)
+constexpr int kMaxRuns = 192;  // visible row runs per attention call, over all its query units
+constexpr int kMaxQUnits = 64; // query units per attention call
 constexpr int kMaxLaneCtas = 1024;
 
-// Visible key rows of one (layer, head) plane: runs of consecutive rows, cut
-// into kBlockN-row tiles; tile_begin[r] is the first tile of run r.
+// Visible key rows of one (layer, head) plane as runs of consecutive rows.
+// Query unit j of a call owns runs [QueryUnits::run_first[j], run_first[j+1]);
+// each run is cut into kBlockN-row tiles, and tile_begin[r] is the first tile
+// of run r among its unit's tiles.
 struct KeyRuns {
   int32_t n_runs;
-  int32_t total_tiles;      // key tiles of one (Q tile, head) item
   int32_t row_begin[kMaxRuns];
   int32_t rows[kMaxRuns];
-  int32_t tile_begin[kMaxRuns + 1];
+  int32_t tile_begin[kMaxRuns];
 };
 
-// Work decomposition.  An item is (Q block qt of kItemRows rows, head h) over
-// all key tiles.  The Q blocks are cut into lanes of `group` consecutive
-// blocks; every lane has `lane_ctas` CTAs, and CTA idx of a lane processes the
-// iterations [idx*per, (idx+1)*per) of its lane's (head, Q block of the lane,
-// key tile) sequence, head major.  CTAs with the same idx in different lanes
-// then read the same K/V tiles at about the same time (L2 reuse).  An item
-// covered by one CTA is written as bf16 directly; an item cut between CTAs is
-// written as fp32 partials (slot item*max_pieces + piece, item = qt*H + h) and
-// merged.
+// The query units of one call (one for the per-unit step, several for a
+// prefill): unit j's queries are rows [j*rows, (j+1)*rows) of q and out, and
+// see tile_start[j+1] - tile_start[j] key tiles.
+struct QueryUnits {
+  int32_t n_units;
+  int32_t rows;                        // query rows per unit (Nq)
+  int32_t tile_start[kMaxQUnits + 1];  // prefix sums of the units' key tiles
+  int32_t run_first[kMaxQUnits + 1];
+};
+
+// Work decomposition.  An item is (query unit j, block qt of kItemRows query
+// rows, head h) over that unit's key tiles.  The blocks are cut into lanes of
+// `group` consecutive blocks; every lane has `lane_ctas` CTAs, and CTA idx of a
+// lane processes the iterations [idx*per, (idx+1)*per) of its lane's sequence
+// (head, block of the lane, query unit, key tile), head major.  CTAs with the
+// same idx in different lanes then read the same K/V tiles at about the same
+// time (L2 reuse).  An item covered by one CTA is written as bf16 directly; an
+// item cut by a CTA boundary is written as fp32 partials and merged.  Only the
+// first and the last item of a CTA's range can be cut, so the partials need two
+// slots per CTA: slot (cta, 0) for its first item, (cta, 1) for its last.
 struct Decomp {
-  int32_t n_qtiles;         // Q blocks of kItemRows rows
-  int32_t group;            // Q blocks per lane
+  int32_t n_qtiles;         // query blocks per unit
+  int32_t group;            // query blocks per lane
   int32_t lanes;
   int32_t lane_ctas;
-  int32_t tiles;            // key tiles per item
+  int32_t tiles;            // key tiles of one (head, block) over all query units (sum over units)
   int32_t heads;
-  int32_t max_pieces;
 };
 
 __host__ __device__ inline int lane_qtiles(const Decomp& d, int lane) {
@@ -52,29 +64,36 @@ __host__ __device__ inline long long lane_work(const Decomp& d, int lane) {
 __host__ __device__ inline long long lane_per(const Decomp& d, int lane) {
   return (lane_work(d, lane) + d.lane_ctas - 1) / d.lane_ctas;
 }
-// First lane iteration of item (qt, h) and the CTAs (lane-local) that cover it.
-__host__ __device__ inline void item_span(const Decomp& d, int qt, int h, int& first_cta, int& pieces) {
-  const int lane = qt / d.group;
+// The CTAs (lane-local) that cover item (j, qt, h), and the partial slot index
+// of its first piece (0 when the item starts exactly at that CTA's range).
+__host__ __device__ inline void item_span(const Decomp& d, const QueryUnits& u, int j, int qt, int h,
+                                          int& lane, int& first_cta, int& pieces, int& first_slot_end) {
+  lane = qt / d.group;
   const int a = qt - lane * d.group;
-  const long long start = ((long long)h * lane_qtiles(d, lane) + a) * d.tiles;
+  const long long start = ((long long)h * lane_qtiles(d, lane) + a) * d.tiles + u.tile_start[j];
+  const int len = u.tile_start[j + 1] - u.tile_start[j];
   const long long per = lane_per(d, lane);
   first_cta = (int)(start / per);
-  pieces = (int)((start + d.tiles - 1) / per) - first_cta + 1;
+  pieces = (int)((start + len - 1) / per) - first_cta + 1;
+  first_slot_end = start == (long long)first_cta * per ? 0 : 1;
+}
+__host__ __device__ inline size_t partial_slot(const Decomp& d, int lane, int cta, int end) {
+  return ((size_t)lane * d.lane_ctas + cta) * 2 + end;
 }
 
 struct AttnParams {
-  int32_t n_query;          // Nq
   int32_t n_heads;          // H
   int32_t plane_k;          // KV-map plane index of head 0's K of this layer
   int32_t plane_v;          // same for V
   float scale_log2;         // log2(e) / sqrt(D)
-  uint16_t* out;            // [Nq][H][D] bf16
-  float* part_o;            // [n_qtiles*H*max_pieces][kItemRows][D] fp32
-  float* part_ml;           // [n_qtiles*H*max_pieces][kItemRows][2] (reference max in log2 units, sum)
+  uint16_t* out;            // [n_units * Nq][H][D] bf16
+  float* part_o;            // [2 * CTAs][kItemRows][D] fp32
+  float* part_ml;           // [2 * CTAs][kItemRows][2] (reference max in log2 units, sum)
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
   int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)
   Decomp dec;
+  QueryUnits qu;
   KeyRuns runs;
 };
 
@@ -85,8 +104,11 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
                              int head_dim, int* ctas, cudaStream_t stream);
-// Chooses the work decomposition of one attention call (defined in ws_api.cu).
-bool decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap);
+// Chooses the work decomposition of one attention call (defined in ws_api.cu):
+// the Q-block lanes together hold one CTA per SM (or `forced` CTAs per lane).
+void decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced);
+// Partial slots a decomposition needs (two per CTA).
+inline int64_t partial_slots(const Decomp& d) { return (int64_t)d.lanes * d.lane_ctas * 2; }
 
 // Merge of the partials of items shared by several CTAs (no-op for the others).
 cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream);

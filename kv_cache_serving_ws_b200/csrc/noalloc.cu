@@ -13,8 +13,10 @@
 // file-scope device array instead of allocated memory.
 //
 // Limits and sharing: the array holds kScratchBytes (48 MiB) on every device
-// that loads this part of the library, until the process exits.  Requests
-// whose partials would not fit are rejected with WS_ERR_UNSUPPORTED.  All
+// that loads this part of the library, until the process exits.  The partials
+// take two slots per CTA (at most one CTA per SM unless the query blocks
+// outnumber the SMs): 39 MB at head_dim 128 on 148 SMs.  Requests whose
+// partials would not fit are rejected with WS_ERR_UNSUPPORTED.  All
 // calls share the array, and it keeps the last call's contents: calls that
 // overlap on the GPU (different streams, or different host threads without
 // ordering) race on it and must be serialised by the caller.  The status word
@@ -66,21 +68,25 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
     return WS_ERR_ALIGN;
   if ((int64_t)n_heads * 2 >= ((int64_t)1 << 31)) return WS_ERR_ARG;
 
-  // one run of visible keys: rows [0, n_keys) of every plane
+  // one query unit, one run of visible keys: rows [0, n_keys) of every plane
   AttnParams p{};
+  p.qu.n_units = 1;
+  p.qu.rows = n_query;
+  p.qu.run_first[0] = 0;
+  p.qu.run_first[1] = 1;
+  p.qu.tile_start[0] = 0;
+  p.qu.tile_start[1] = (n_keys + kBlockN - 1) / kBlockN;
   p.runs.n_runs = 1;
   p.runs.row_begin[0] = 0;
   p.runs.rows[0] = n_keys;
   p.runs.tile_begin[0] = 0;
-  p.runs.tile_begin[1] = (n_keys + kBlockN - 1) / kBlockN;
-  p.runs.total_tiles = p.runs.tile_begin[1];
 
-  // scratch layout: [status | part_ml | part_o]; slots sized for this call
+  // scratch layout: [status | part_ml | part_o], two partial slots per CTA
   const int n_qtiles = (n_query + kItemRows - 1) / kItemRows;
+  decompose(p.dec, n_qtiles, n_heads, p.qu.tile_start[1], 0);
+  const size_t slots = (size_t)partial_slots(p.dec);
   const size_t slot_bytes = (size_t)kItemRows * (head_dim + 2) * sizeof(float);
-  const int64_t slot_cap = (int64_t)((kScratchBytes - kStatusBytes) / slot_bytes);
-  if (!decompose(p.dec, n_qtiles, n_heads, p.runs.total_tiles, 0, slot_cap)) return WS_ERR_UNSUPPORTED;
-  const size_t slots = (size_t)n_qtiles * n_heads * p.dec.max_pieces;
+  if (kStatusBytes + slots * slot_bytes > kScratchBytes) return WS_ERR_UNSUPPORTED;
 
   void* base = nullptr;
   const int st = scratch_address(&base);
@@ -90,7 +96,6 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   p.part_ml = reinterpret_cast<float*>(b + kStatusBytes);
   p.part_o = reinterpret_cast<float*>(b + kStatusBytes + slots * kItemRows * 2 * sizeof(float));
 
-  p.n_query = n_query;
   p.n_heads = n_heads;
   p.plane_k = 0;
   p.plane_v = n_heads;
@@ -108,8 +113,8 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   bool any_split = false;
   for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
     for (int h = 0; h < n_heads && !any_split; ++h) {
-      int c_first, pieces;
-      item_span(p.dec, qt, h, c_first, pieces);
+      int lane, c_first, pieces, end0;
+      item_span(p.dec, p.qu, 0, qt, h, lane, c_first, pieces, end0);
       any_split = pieces > 1;
     }
   if (any_split && launch_merge(p, head_dim, stream) != cudaSuccess) return WS_ERR_CUDA;

@@ -16,13 +16,12 @@
 
 using namespace ws;
 
-// Work decomposition of one attention call (see Decomp in kernels.cuh).  The Q
-// tiles are grouped into lanes so that the lanes together hold one CTA per SM;
-// the group size minimises the iterations of the busiest CTA (ties: the
-// smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
-// iterations.  `forced` > 0 fixes the CTAs per lane.  Returns false when the
-// partial slots would not fit the workspace even with one CTA per lane.
-bool ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int64_t slot_cap) {
+// Work decomposition of one attention call (see Decomp in kernels.cuh).  The
+// query blocks are grouped into lanes so that the lanes together hold one CTA
+// per SM; the group size minimises the iterations of the busiest CTA (ties:
+// the smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
+// iterations.  `forced` > 0 fixes the CTAs per lane.
+void ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced) {
   const int sms = sm_count();
   d.n_qtiles = n_qtiles;
   d.heads = heads;
@@ -47,17 +46,7 @@ bool ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, in
   }
   d.group = best_g;
   d.lanes = (n_qtiles + best_g - 1) / best_g;
-  for (int cpl = best_cpl;; cpl = std::max(1, cpl / 2)) {
-    d.lane_ctas = cpl;
-    long long min_per = -1;
-    for (int ln = 0; ln < d.lanes; ++ln) {
-      const long long per = lane_per(d, ln);
-      if (min_per < 0 || per < min_per) min_per = per;
-    }
-    d.max_pieces = (int)((tiles + min_per - 1) / min_per) + 1;
-    if ((int64_t)n_qtiles * heads * d.max_pieces <= slot_cap) return true;
-    if (cpl == 1) return false;
-  }
+  d.lane_ctas = best_cpl;
 }
 
 struct EventPool {
@@ -183,6 +172,129 @@ void free_all(ws_cache* h) {
 
 }  // namespace
 
+namespace {
+
+// Attention of the query units u_first .. u_first+n-1 at `layer` (one unit for
+// the per-unit step, several for a prefill).  Writes each unit's k_new/v_new
+// into its latent rows, plans each unit's visible runs, launches the kernel
+// and, when a head's key range was cut between CTAs, the merge.
+int attention_impl(ws_cache_t* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || u_first < 0 || n < 1) return WS_ERR_ARG;
+  if (n > kMaxQUnits) return WS_ERR_UNSUPPORTED;
+  if (!q || !k_new || !v_new || !out) return WS_ERR_ARG;
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return WS_ERR_ALIGN;
+  const int64_t u_last = u_first + n - 1;
+  if (h->newest < 0 || u_last > h->newest) return WS_ERR_NOT_READY;
+  if (u_last < h->newest) return WS_ERR_UNIT_ORDER;
+  const int H = h->cfg.n_heads, D = h->cfg.head_dim, L = h->cfg.n_layers, U = h->cfg.history_units;
+  // every query unit must be resident, and no unit of any query window evicted
+  for (int64_t u = u_first; u <= u_last; ++u) {
+    const int st = resident(h, u);
+    if (st != WS_OK) return st;
+  }
+  // units before the first query unit lie in some query window; one whose slot
+  // now holds a newer unit (a later query unit of a long prefill) is gone
+  for (int64_t u = std::max<int64_t>(0, u_first - U); u < u_first; ++u)
+    if (h->slot_unit[(size_t)(u % h->C)] > u) return WS_ERR_EVICTED;
+
+  // plan first (pure host work), so that an unsupported layout changes nothing
+  std::vector<uint8_t> ready(h->latent_ready);
+  for (int64_t u = u_first; u <= u_last; ++u) ready[(size_t)(u % h->C) * L + layer] = 1;
+  AttnParams p{};
+  p.qu.n_units = n;
+  p.qu.rows = h->Nq;
+  int runs = 0, tiles = 0;
+  int64_t keys = 0;
+  for (int j = 0; j < n; ++j) {
+    p.qu.run_first[j] = runs;
+    p.qu.tile_start[j] = tiles;
+    int32_t nr = 0;
+    const int st = plan_runs(h->cfg, h->slot_unit.data(), ready.data(), layer, u_first + j, p.runs.row_begin + runs,
+                             p.runs.rows + runs, kMaxRuns - runs, &nr);
+    if (st != WS_OK) return st;
+    int t = 0;
+    for (int r = runs; r < runs + nr; ++r) {
+      p.runs.tile_begin[r] = t;
+      t += (p.runs.rows[r] + kBlockN - 1) / kBlockN;
+      keys += p.runs.rows[r];
+    }
+    runs += nr;
+    tiles += t;
+  }
+  p.qu.run_first[n] = runs;
+  p.qu.tile_start[n] = tiles;
+  p.runs.n_runs = runs;
+
+  const int n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
+  decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas);
+  while (partial_slots(p.dec) > h->slot_cap && p.dec.lane_ctas > 1)
+    decompose(p.dec, n_qtiles, H, tiles, std::max(1, p.dec.lane_ctas / 2));
+  if (partial_slots(p.dec) > h->slot_cap) return WS_ERR_UNSUPPORTED;
+  bool any_split = false;
+  for (int j = 0; j < n && !any_split; ++j)
+    for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
+      for (int hh = 0; hh < H && !any_split; ++hh) {
+        int lane, c_first, pieces, end0;
+        item_span(p.dec, p.qu, j, qt, hh, lane, c_first, pieces, end0);
+        any_split = pieces > 1;
+      }
+
+  CUtensorMap q_map;
+  if (encode_q_map(&q_map, q, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
+
+  // 1. the query units' latent K/V of this layer into their slots
+  const size_t unit_elems = (size_t)h->Nq * H * D;
+  for (int j = 0; j < n; ++j) {
+    const size_t slot = (size_t)((u_first + j) % h->C);
+    AppendParams a{};
+    a.src_k = k_new + j * unit_elems;
+    a.src_v = v_new + j * unit_elems;
+    a.cache = h->kv;
+    a.n_layers = 1;
+    a.layer0 = layer;
+    a.n_tokens = h->Nq;
+    a.n_heads = H;
+    a.head_dim = D;
+    a.plane_rows = (int64_t)h->C * h->T;
+    a.row0 = (int64_t)slot * h->T + h->cfg.n_cond;
+    cudaEvent_t* ev = h->profiling ? h->ev_lat.next() : nullptr;
+    if (ev) cudaEventRecord(ev[0], stream);
+    if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
+    if (ev) cudaEventRecord(ev[1], stream);
+    h->latent_ready[slot * L + layer] = 1;
+  }
+
+  // 2. attention (+ merge of the partials of cut items)
+  p.n_heads = H;
+  p.plane_k = (layer * 2 + 0) * H;
+  p.plane_v = (layer * 2 + 1) * H;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.out = out;
+  p.part_o = h->part_o;
+  p.part_ml = h->part_ml;
+  p.status = h->d_status;
+  p.timeout_ns = h->timeout_ns;
+  p.debug_skip_v_tile = h->debug_skip_v_tile;
+  cudaEvent_t* ev = h->profiling ? h->ev_attn.next() : nullptr;
+  if (ev) cudaEventRecord(ev[0], stream);
+  int ctas = 0;
+  if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (ev) cudaEventRecord(ev[1], stream);
+  if (any_split) {
+    ev = h->profiling ? h->ev_comb.next() : nullptr;
+    if (ev) cudaEventRecord(ev[0], stream);
+    if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
+    if (ev) cudaEventRecord(ev[1], stream);
+  }
+  h->last_split = p.dec.lane_ctas;
+  h->last_ctas = ctas;
+  h->last_keys = keys;
+  return WS_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* ws_status_string(int status) {
@@ -228,9 +340,10 @@ int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t s
   const int L = cfg->n_layers, H = cfg->n_heads, D = cfg->head_dim;
   const int64_t rows = (int64_t)h->C * h->T;
   h->kv_bytes = (size_t)L * 2 * H * rows * D * 2;
-  // partial slots: items x (ceil(SMs / H) + 1) bounds every automatic decomposition
+  // partial slots: two per CTA; an automatic decomposition has at most one CTA
+  // per SM (more only when the query blocks outnumber the SMs)
   const int64_t n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
-  h->slot_cap = n_qtiles * H * ((sm_count() + H - 1) / H + 1);
+  h->slot_cap = 2 * std::max<int64_t>(sm_count(), n_qtiles);
   const size_t part_o_bytes = (size_t)h->slot_cap * kItemRows * D * 4;
   const size_t part_ml_bytes = (size_t)h->slot_cap * kItemRows * 2 * 4;
   h->ws_bytes = part_o_bytes + part_ml_bytes;
@@ -308,90 +421,12 @@ int ws_cache_append(ws_cache_t* h, int64_t unit, int seg, const uint16_t* k_slic
 
 int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q, const uint16_t* k_new,
                       const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
-  if (!h || layer < 0 || layer >= h->cfg.n_layers || unit < 0) return WS_ERR_ARG;
-  if (!q || !k_new || !v_new || !out) return WS_ERR_ARG;
-  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return WS_ERR_ALIGN;
-  if (h->newest < 0 || unit > h->newest) return WS_ERR_NOT_READY;
-  if (unit < h->newest) return WS_ERR_UNIT_ORDER;
-  const int H = h->cfg.n_heads, D = h->cfg.head_dim, L = h->cfg.n_layers;
-  const size_t slot = (size_t)(unit % h->C);
+  return attention_impl(h, layer, unit, 1, q, k_new, v_new, out, stream);
+}
 
-  // plan first (pure host work), so that an unsupported layout changes nothing
-  std::vector<uint8_t> ready(h->latent_ready);
-  ready[slot * L + layer] = 1;
-  AttnParams p{};
-  int32_t n_runs = 0;
-  int st = plan_runs(h->cfg, h->slot_unit.data(), ready.data(), layer, unit, p.runs.row_begin, p.runs.rows,
-                     kMaxRuns, &n_runs);
-  if (st != WS_OK) return st;
-  p.runs.n_runs = n_runs;
-  int tiles = 0;
-  int64_t keys = 0;
-  for (int r = 0; r < n_runs; ++r) {
-    p.runs.tile_begin[r] = tiles;
-    tiles += (p.runs.rows[r] + kBlockN - 1) / kBlockN;
-    keys += p.runs.rows[r];
-  }
-  p.runs.tile_begin[n_runs] = tiles;
-  p.runs.total_tiles = tiles;
-
-  CUtensorMap q_map;
-  if (encode_q_map(&q_map, q, D, H, h->Nq) != 0) return WS_ERR_CUDA;
-
-  // 1. the current unit's latent K/V of this layer into its slot
-  AppendParams a{};
-  a.src_k = k_new;
-  a.src_v = v_new;
-  a.cache = h->kv;
-  a.n_layers = 1;
-  a.layer0 = layer;
-  a.n_tokens = h->Nq;
-  a.n_heads = H;
-  a.head_dim = D;
-  a.plane_rows = (int64_t)h->C * h->T;
-  a.row0 = (int64_t)slot * h->T + h->cfg.n_cond;
-  cudaEvent_t* ev = h->profiling ? h->ev_lat.next() : nullptr;
-  if (ev) cudaEventRecord(ev[0], stream);
-  if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
-  if (ev) cudaEventRecord(ev[1], stream);
-  h->latent_ready[slot * L + layer] = 1;
-
-  // 2. attention (+ merge of split partials)
-  p.n_query = h->Nq;
-  p.n_heads = H;
-  const int n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
-  if (!decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas, h->slot_cap)) return WS_ERR_UNSUPPORTED;
-  bool any_split = false;
-  for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
-    for (int hh = 0; hh < H && !any_split; ++hh) {
-      int c_first, pieces;
-      item_span(p.dec, qt, hh, c_first, pieces);
-      any_split = pieces > 1;
-    }
-  p.plane_k = (layer * 2 + 0) * H;
-  p.plane_v = (layer * 2 + 1) * H;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  p.out = out;
-  p.part_o = h->part_o;
-  p.part_ml = h->part_ml;
-  p.status = h->d_status;
-  p.timeout_ns = h->timeout_ns;
-  p.debug_skip_v_tile = h->debug_skip_v_tile;
-  ev = h->profiling ? h->ev_attn.next() : nullptr;
-  if (ev) cudaEventRecord(ev[0], stream);
-  int ctas = 0;
-  if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
-  if (ev) cudaEventRecord(ev[1], stream);
-  if (any_split) {
-    ev = h->profiling ? h->ev_comb.next() : nullptr;
-    if (ev) cudaEventRecord(ev[0], stream);
-    if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
-    if (ev) cudaEventRecord(ev[1], stream);
-  }
-  h->last_split = p.dec.lane_ctas;
-  h->last_ctas = ctas;
-  h->last_keys = keys;
-  return WS_OK;
+int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n_units, const uint16_t* q,
+                         const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  return attention_impl(h, layer, unit_first, n_units, q, k_new, v_new, out, stream);
 }
 
 int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {

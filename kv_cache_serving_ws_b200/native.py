@@ -70,6 +70,7 @@ def _declare(lib):
         "ws_cache_destroy": (C.c_int, [_P]),
         "ws_cache_append": (C.c_int, [_P, i64, C.c_int, _P, _P, _P]),
         "ws_unit_attention": (C.c_int, [_P, C.c_int, i64, _P, _P, _P, _P, _P]),
+        "ws_prefill_attention": (C.c_int, [_P, C.c_int, i64, i32, _P, _P, _P, _P, _P]),
         "ws_flow_step": (C.c_int, [_P, _P, C.c_float, i64, _P]),
         "ws_cache_read": (C.c_int, [_P, C.c_int, i64, C.c_int, _P, _P, _P]),
         "ws_cache_slot_table": (C.c_int, [_P, C.POINTER(i64)]),
@@ -185,6 +186,11 @@ def ws_cache_append(h, unit, seg, k_slice, v_slice, stream=None, check=True):
 def ws_unit_attention(h, layer, unit, q, k_new, v_new, out, stream=None, check=True):
     return _done(lib().ws_unit_attention(h, layer, unit, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
                                          _stream(stream)), "ws_unit_attention", check)
+
+
+def ws_prefill_attention(h, layer, unit_first, n_units, q, k_new, v_new, out, stream=None, check=True):
+    return _done(lib().ws_prefill_attention(h, layer, unit_first, n_units, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                            _ptr(out), _stream(stream)), "ws_prefill_attention", check)
 
 
 def ws_flow_step(x, v, dt, n=None, stream=None, check=True):

@@ -55,6 +55,8 @@ ERR_OOM = -3
 ERR_UNIT_ORDER = -4
 ERR_EVICTED = -5
 ERR_NOT_READY = -6
+ERR_UNSUPPORTED = -9
+MAX_QUERY_UNITS = 64
 
 SEG_COND = 0
 SEG_LATENT = 1
@@ -299,6 +301,46 @@ class UnitCache:
         rec.lat_v[layer] = np.array(v_new_bits, dtype=np.uint16)
         k, v, _ = self.visible_kv(layer, unit)
         return OK, attention_rows(bf16_to_f64(q_bits), k, v, rows=rows, heads=heads)
+
+
+    def prefill_attention(self, layer: int, unit_first: int, n_units: int, q_bits, k_new_bits, v_new_bits,
+                          rows=None, heads=None):
+        """Several consecutive query units at once (a prompt prefill): write each
+        unit's latent K/V of ``layer``, then every query unit attends over its own
+        window -- block-causal across units.  q, k_new, v_new: [n, Nq, H, D].
+
+        Every query unit must be resident, the last one the newest, and no unit
+        inside a query window may have been overwritten.
+        Returns (status, out [n, rows, heads, D] float64)."""
+        c = self.cfg
+        shape = (n_units, c.n_query, c.n_heads, c.head_dim)
+        if not (0 <= layer < c.n_layers) or unit_first < 0 or n_units < 1:
+            return ERR_ARG, None
+        if n_units > MAX_QUERY_UNITS:
+            return ERR_UNSUPPORTED, None
+        if any(np.shape(a) != shape for a in (q_bits, k_new_bits, v_new_bits)):
+            return ERR_ARG, None
+        u_last = unit_first + n_units - 1
+        if u_last > self.newest:
+            return ERR_NOT_READY, None
+        if u_last < self.newest:
+            return ERR_UNIT_ORDER, None
+        for u in range(unit_first, u_last + 1):
+            st = self._resident(u)
+            if st != OK:
+                return st, None
+        for u in range(max(0, unit_first - self.cfg.history_units), unit_first):
+            if self.slot_unit[self.slot(u)] > u:
+                return ERR_EVICTED, None
+        for j in range(n_units):
+            rec = self.units[unit_first + j]
+            rec.lat_k[layer] = np.array(k_new_bits[j], dtype=np.uint16)
+            rec.lat_v[layer] = np.array(v_new_bits[j], dtype=np.uint16)
+        outs = []
+        for j in range(n_units):
+            k, v, _ = self.visible_kv(layer, unit_first + j)
+            outs.append(attention_rows(bf16_to_f64(q_bits[j]), k, v, rows=rows, heads=heads))
+        return OK, np.stack(outs)
 
 
 def attention_flops(n_query: int, n_keys: int, n_heads: int, head_dim: int) -> float:

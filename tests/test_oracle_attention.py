@@ -295,3 +295,68 @@ def test_error_rules():
     assert cache.read(0, 0, orc.SEG_COND)[0] == orc.ERR_EVICTED
     assert cache.read(0, 4, orc.SEG_COND)[0] == orc.OK
     assert cache.append(-1, orc.SEG_COND, zc, zc) == orc.ERR_ARG
+
+
+@pytest.mark.parametrize("U,n_prior,n_units", [(3, 0, 4), (5, 2, 4), (4, 1, 3), (2, 3, 1), (2, 3, 3), (0, 1, 3)])
+def test_prefill_equals_full_recomputation_per_query_unit(U, n_prior, n_units):
+    """A multi-unit query: every query unit's rows against the dense block-causal
+    mask over the whole sequence (pure-Python brute force)."""
+    cfg = _cfg(history_units=U)
+    cache = orc.UnitCache(cfg)
+    prior = list(range(n_prior))
+    _fill(cache, cfg, prior + [n_prior], commit=True)           # committed history; unit n_prior: COND only
+    qunits = list(range(n_prior, n_prior + n_units))
+    for u in qunits[1:]:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        assert cache.append(u, orc.SEG_COND, _bits(1, synth.KIND_COND_K, cs, u),
+                            _bits(1, synth.KIND_COND_V, cs, u)) == orc.OK
+    layer = 1
+    qs = (n_units, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q = _bits(6, synth.KIND_Q, qs, n_prior, layer)
+    kn = _bits(6, synth.KIND_K_NEW, qs, n_prior, layer)
+    vn = _bits(6, synth.KIND_V_NEW, qs, n_prior, layer)
+    st, out = cache.prefill_attention(layer, n_prior, n_units, q, kn, vn)
+    # a unit inside some query window is gone once a later unit took its slot
+    # (slot reuse after C = U + 1 units): a query unit itself, or a prior unit
+    # of the first query unit's window
+    u_last = n_prior + n_units - 1
+    gone = n_units > cfg.slots or any(u + cfg.slots <= u_last for u in prior if u >= n_prior - U)
+    if gone:
+        assert st == orc.ERR_EVICTED
+        return
+    assert st == orc.OK
+    seq = []
+    for uu in prior + qunits:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        ck = orc.bf16_to_f64(_bits(1, synth.KIND_COND_K, cs, uu))[layer]
+        cv = orc.bf16_to_f64(_bits(1, synth.KIND_COND_V, cs, uu))[layer]
+        seq += [(uu, "cond", ck[t], cv[t]) for t in range(cfg.n_cond)]
+        if uu in qunits:
+            j = uu - n_prior
+            lk, lv = orc.bf16_to_f64(kn[j]), orc.bf16_to_f64(vn[j])
+        else:
+            ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+            lk = orc.bf16_to_f64(_bits(1, synth.KIND_COMMIT_K, ls, uu))[layer]
+            lv = orc.bf16_to_f64(_bits(1, synth.KIND_COMMIT_V, ls, uu))[layer]
+        seq += [(uu, "latent", lk[t], lv[t]) for t in range(cfg.n_query)]
+    for j, uq in enumerate(qunits):
+        want = _brute_force(cfg, seq, uq, layer, orc.bf16_to_f64(q[j]))
+        assert np.max(np.abs(out[j] - want)) <= 1e-12, uq
+
+
+def test_prefill_error_rules():
+    cfg = _cfg(history_units=3)                                  # C = 4
+    cache = orc.UnitCache(cfg)
+    _fill(cache, cfg, [0, 1, 2, 3], commit=False)
+    qs = lambda n: np.zeros((n, cfg.n_query, cfg.n_heads, cfg.head_dim), np.uint16)
+    assert cache.prefill_attention(0, 0, 4, qs(4), qs(4), qs(4))[0] == orc.OK           # from scratch
+    assert cache.prefill_attention(0, 1, 3, qs(3), qs(3), qs(3))[0] == orc.OK           # unit 0 still resident
+    assert cache.prefill_attention(0, 2, 3, qs(3), qs(3), qs(3))[0] == orc.ERR_NOT_READY # unit 4 not there yet
+    assert cache.prefill_attention(0, 1, 2, qs(2), qs(2), qs(2))[0] == orc.ERR_UNIT_ORDER
+    assert cache.prefill_attention(0, 1, 3, qs(4), qs(3), qs(3))[0] == orc.ERR_ARG       # shape
+    assert cache.prefill_attention(0, 0, 65, qs(65), qs(65), qs(65))[0] == orc.ERR_UNSUPPORTED
+    _fill(cache, cfg, [4], commit=False)                         # unit 4 takes unit 0's slot
+    assert cache.prefill_attention(0, 1, 4, qs(4), qs(4), qs(4))[0] == orc.ERR_EVICTED   # 0 in unit 1's window
+    assert cache.prefill_attention(0, 3, 2, qs(2), qs(2), qs(2))[0] == orc.ERR_EVICTED   # 0 in unit 3's window
+    assert cache.prefill_attention(0, 4, 1, qs(1), qs(1), qs(1))[0] == orc.OK            # window 1..4
+    assert cache.prefill_attention(0, 0, 5, qs(5), qs(5), qs(5))[0] == orc.ERR_EVICTED   # query unit 0 gone
