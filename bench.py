@@ -567,6 +567,151 @@ def run_prefill(args):
         sys.exit(1)
 
 
+def percentiles(xs):
+    a = sorted(xs)
+
+    def pct(p):
+        i = min(len(a) - 1, max(0, int(round(p / 100.0 * (len(a) - 1)))))
+        return round(a[i], 3)
+    return {"p50": pct(50), "p99": pct(99), "max": round(a[-1], 3), "min": round(a[0], 3),
+            "mean": round(statistics.fmean(a), 3)}
+
+
+def run_schedule(args):
+    """Per-unit schedule of the whole unit (conditioning append, 40 layers x 4 Euler
+    steps of attention, commit), units back to back and paced at the stream's 160 ms
+    cadence.  Direct calls (~490 launches per unit) against the unit program (one CUDA
+    graph per unit, updated in place).  Reports per-unit device time percentiles, the
+    host time the program spends recording a unit, and, paced, the latency from a
+    unit's release (its conditioning slice copied from pinned host memory) to its
+    completion, with the backlog's growth per unit when a unit outlasts 160 ms."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200 import synth
+    from kv_cache_serving_ws_b200.workloads import FULL, FULL32, GpuSession, key
+    period_s = 0.160
+    n = args.units
+    for w in (FULL32, FULL):
+        L, S = w.n_layers, w.steps
+        g = GpuSession(w)
+        dev = g.dev
+        bf = torch.bfloat16
+        qs = (w.n_query, w.n_heads, w.head_dim)
+        n_lat = w.n_query * w.n_heads * w.head_dim
+        q_all = torch.empty((S, L) + qs, dtype=bf, device=dev)
+        kn_all, vn_all = torch.empty_like(q_all), torch.empty_like(q_all)
+        for s in range(S):
+            for l in range(L):
+                g.fill(q_all[s, l], key(w, synth.KIND_Q, w.unit, l, s))
+                g.fill(kn_all[s, l], key(w, synth.KIND_K_NEW, w.unit, l, s))
+                g.fill(vn_all[s, l], key(w, synth.KIND_V_NEW, w.unit, l, s))
+        vel = torch.empty((S, n_lat), dtype=bf, device=dev)
+        for s in range(S):
+            g.fill(vel[s], key(w, synth.KIND_VEL, w.unit, 0, s))
+        x = torch.empty(n_lat, dtype=bf, device=dev)
+        g.fill(x, key(w, synth.KIND_X, w.unit))
+        out = torch.empty(qs, dtype=bf, device=dev)
+        ck, cv = torch.empty_like(g.cond_k), torch.empty_like(g.cond_v)
+        g.fill(ck, key(w, synth.KIND_COND_K, w.unit))
+        g.fill(cv, key(w, synth.KIND_COND_V, w.unit))
+        commit_k, commit_v = g.commit_buffers()
+        for u in range(w.unit):
+            g.append_cond(u)
+            g.commit(u)
+        g.fill(commit_k, key(w, synth.KIND_COMMIT_K, w.unit))
+        g.fill(commit_v, key(w, synth.KIND_COMMIT_V, w.unit))
+        host_ck, host_cv = ck.cpu().pin_memory(), cv.cpu().pin_memory()
+        torch.cuda.synchronize()
+        nxt = [w.unit]
+
+        def direct():
+            u = nxt[0]
+            ws.ws_cache_append(g.h, u, ws.WS_SEG_COND, ck, cv)
+            for s in range(S):
+                for l in range(L):
+                    ws.ws_unit_attention(g.h, l, u, q_all[s, l], kn_all[s, l], vn_all[s, l], out)
+                ws.ws_flow_step(x, vel[s], w.dt)
+            ws.ws_cache_append(g.h, u, ws.WS_SEG_LATENT, commit_k, commit_v)
+            nxt[0] = u + 1
+
+        _, prog = ws.ws_unit_graph_create(g.h, S, w.dt, ck, cv, q_all, kn_all, vn_all, out, x, vel, commit_k,
+                                          commit_v, out_per_call=False)
+
+        def graph():
+            ws.ws_unit_graph_launch(prog, nxt[0])
+            nxt[0] += 1
+
+        def back_to_back(fn):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
+            t0 = time.perf_counter()
+            ev[0].record()
+            for i in range(n):
+                fn()
+                ev[i + 1].record()
+            t_host = time.perf_counter() - t0
+            torch.cuda.synchronize()
+            per = [ev[i].elapsed_time(ev[i + 1]) for i in range(n)]
+            return per, t_host * 1e3 / n
+
+        with ClockSampler(0) as clk:
+            per_direct, host_direct = back_to_back(direct)
+            s0 = ws.ws_unit_graph_get_stats(prog)
+            per_graph, host_graph = back_to_back(graph)
+            s1 = ws.ws_unit_graph_get_stats(prog)
+
+            # paced: unit k is released at t0 + k * 160 ms with its conditioning slice
+            torch.cuda.synchronize()
+            pending, lat = [], []
+            t0 = time.perf_counter() + 0.02
+            k = 0
+            while k < n or pending:
+                now = time.perf_counter()
+                while pending and pending[0][1].query():
+                    lat.append((now - pending[0][0]) * 1e3)
+                    pending.pop(0)
+                if k < n and now >= t0 + k * period_s:
+                    ck.copy_(host_ck, non_blocking=True)
+                    cv.copy_(host_cv, non_blocking=True)
+                    graph()
+                    e = torch.cuda.Event()
+                    e.record()
+                    pending.append((t0 + k * period_s, e))
+                    k += 1
+                    continue
+                time.sleep(0.0002)
+        st = ws.ws_sync(g.h, check=False)
+        ws.ws_unit_graph_destroy(prog)
+        slope = 0.0
+        if len(lat) > 1:
+            xs = list(range(len(lat)))
+            mx, my = statistics.fmean(xs), statistics.fmean(lat)
+            slope = sum((a - mx) * (b - my) for a, b in zip(xs, lat)) / sum((a - mx) ** 2 for a in xs)
+        upd = s1["updates"] - s0["updates"]
+        inst = s1["instantiations"] - s0["instantiations"]
+        flops_unit = w.flops_per_call() * L * S
+        print(json.dumps({
+            "mode": "schedule", "workload": w.name, "units": n, "unit_budget_ms": period_s * 1e3,
+            "tflop_per_unit": round(flops_unit / 1e12, 2),
+            "direct": {"unit_ms": percentiles(per_direct), "host_ms_per_unit": round(host_direct, 3),
+                       "launches_per_unit": 2 + L * S * 3 + S},
+            "graph": {"unit_ms": percentiles(per_graph), "host_ms_per_unit": round(host_graph, 3),
+                      "record_ms_per_unit": round((s1["record_ms"] - s0["record_ms"]) / max(1, n + 3), 3),
+                      "kernel_nodes": s1["nodes"], "updates_in_place": upd, "instantiations": inst,
+                      "TFLOP/s_p50": round(flops_unit / percentiles(per_graph)["p50"] / 1e9, 1)},
+            "paced_160ms": {"latency_ms": percentiles(lat), "backlog_growth_ms_per_unit": round(slope, 2),
+                            "units_over_budget": sum(1 for v in lat if v > period_s * 1e3)},
+            "clocks": clk.summary(), "status": ws.status_string(st)}), flush=True)
+        del q_all, kn_all, vn_all
+        g.close()
+        torch.cuda.empty_cache()
+        if st != ws.WS_OK:
+            sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -580,12 +725,18 @@ def main():
     ap.add_argument("--calls", type=int, default=3)
     ap.add_argument("--prefill", action="store_true", help="time a multi-unit prompt prefill instead")
     ap.add_argument("--prefill-units", type=int, default=64)
+    ap.add_argument("--schedule", action="store_true",
+                    help="per-unit schedule: direct calls vs the unit program, back to back and paced at 160 ms")
+    ap.add_argument("--units", type=int, default=24)
     args = ap.parse_args()
     if args.case:
         run_case(args)
         return
     if args.prefill:
         run_prefill(args)
+        return
+    if args.schedule:
+        run_schedule(args)
         return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -293,6 +293,86 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit,
 int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query,
                          int32_t n_keys, int32_t n_heads, int32_t head_dim, cudaStream_t stream);
 
+/*
+ * Unit program -- the whole device work of one streaming unit, recorded once
+ * as a CUDA graph and replayed per unit.  One unit is:
+ *   ws_cache_append(unit, WS_SEG_COND, cond_k, cond_v);
+ *   for s in 0..S-1:  for l in 0..L-1:
+ *       ws_unit_attention(l, unit, q[s][l], k_new[s][l], v_new[s][l], out[s][l]);
+ *     ws_flow_step(x, vel[s], dt, n_latent);
+ *   ws_cache_append(unit, WS_SEG_LATENT, commit_k, commit_v);
+ * with exactly the arithmetic, the host bookkeeping and the error rules of those
+ * calls.  The performer has to finish this work inside every 160 ms unit, and
+ * the service overlaps the units' stages (remio.ai, section
+ * 思考者与执行者的分工掩盖了更高分辨率的成本).  A graph launch replaces the unit's
+ * ~490 stream launches by one, so the host can run ahead by whole units and the
+ * kernels start without per-launch host gaps.
+ *
+ * ws_unit_io: device pointers, 16-byte aligned, owned by the caller, fixed for
+ * the life of the program (the graph holds them); their contents may change
+ * between launches.
+ *   cond_k, cond_v      [L][Nc][H][D]   thinker's slice of the unit
+ *   q, k_new, v_new     [S][L][Nq][H][D] per step and layer
+ *   out                 [S][L][Nq][H][D] if out_per_call, else one [Nq][H][D]
+ *                       buffer that every call overwrites
+ *   x                   [n_latent]       latent, updated in place by each step
+ *   vel                 [S][n_latent]    velocity of each step
+ *   commit_k, commit_v  [L][Nq][H][D]   committed K/V of the unit
+ */
+typedef struct {
+  int32_t n_steps;              /* S >= 1 */
+  int32_t out_per_call;         /* 1: out is [S][L][Nq][H][D]; 0: one [Nq][H][D] buffer */
+  float dt;
+  int64_t n_latent;             /* >= 0 */
+  const uint16_t* cond_k;
+  const uint16_t* cond_v;
+  const uint16_t* q;
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* out;
+  uint16_t* x;
+  const uint16_t* vel;
+  const uint16_t* commit_k;
+  const uint16_t* commit_v;
+} ws_unit_io;
+
+typedef struct ws_unit_graph ws_unit_graph_t;   /* opaque */
+
+/* Create a unit program over cache h (which must outlive it).  Records nothing
+ * yet.  Errors: WS_ERR_ARG (NULL, S < 1, n_latent < 0), WS_ERR_ALIGN,
+ * WS_ERR_OOM, WS_ERR_CUDA. */
+int ws_unit_graph_create(ws_unit_graph_t** out, ws_cache_t* h, const ws_unit_io* io);
+
+/*
+ * ws_unit_graph_launch -- enqueue unit `unit` on `stream` as one graph launch.
+ * The unit's calls are recorded on a capture stream of the program (validating
+ * every argument and updating the ring bookkeeping as the direct calls would),
+ * the recorded graph refreshes the program's executable graph in place
+ * (cudaGraphExecUpdate; a new instantiation only when the launch structure
+ * changed), and the executable graph is launched.  In steady state the
+ * recorded launches differ from unit to unit only in the unit's slot rows.
+ * Errors: those of the recorded calls; on an error nothing is launched and the
+ * cache's bookkeeping is left as before the call.  The program's executable
+ * graph is shared by its launches: calls on different streams must be ordered
+ * by the caller.
+ */
+int ws_unit_graph_launch(ws_unit_graph_t* g, int64_t unit, cudaStream_t stream);
+
+/* Counters of a program: launches, instantiations (structure changed) and
+ * in-place updates, and the host time spent recording + updating (ms). */
+typedef struct {
+  int64_t launches;
+  int64_t instantiations;
+  int64_t updates;
+  int64_t nodes;                /* kernel launches in the last recorded unit */
+  double record_ms;             /* host time in capture + update, summed */
+} ws_unit_graph_stats;
+
+int ws_unit_graph_get_stats(const ws_unit_graph_t* g, ws_unit_graph_stats* out);
+
+/* Destroy a program (synchronises its pending launches first). */
+int ws_unit_graph_destroy(ws_unit_graph_t* g);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,0 +1,80 @@
+// Host-side state of a cache handle, shared by the C-ABI translation units
+// (ws_api.cu: cache, attention and Euler entry points; unit_graph.cu: the
+// captured unit program).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <vector>
+
+#include "../../include/ws.h"
+#include "kernels.cuh"
+
+struct EventPool {
+  std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 end
+  int used = 0;
+  int64_t launches = 0;
+  double ms = 0.0;
+  void create(int pairs) {
+    ev.resize(2 * pairs);
+    for (auto& e : ev) cudaEventCreate(&e);
+    used = 0;
+  }
+  void destroy() {
+    for (auto& e : ev) cudaEventDestroy(e);
+    ev.clear();
+  }
+  void flush() {
+    for (int i = 0; i < used; ++i) {
+      cudaEventSynchronize(ev[2 * i + 1]);
+      float t = 0.f;
+      if (cudaEventElapsedTime(&t, ev[2 * i], ev[2 * i + 1]) == cudaSuccess) ms += t;
+    }
+    launches += used;
+    used = 0;
+  }
+  cudaEvent_t* next() {
+    if (ev.empty()) return nullptr;
+    if (2 * used >= (int)ev.size()) flush();
+    return &ev[2 * (used++)];
+  }
+};
+
+struct ws_cache {
+  ws_cache_config cfg{};
+  int device = 0;
+  int C = 0, T = 0, Nq = 0;
+  int64_t newest = -1;
+  std::vector<int64_t> slot_unit;     // C
+  std::vector<uint8_t> latent_ready;  // C * L
+  uint16_t* kv = nullptr;
+  size_t kv_bytes = 0;
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  size_t ws_bytes = 0;
+  int* d_status = nullptr;
+  CUtensorMap kv_map;
+  int force_lane_ctas = 0;
+  int64_t slot_cap = 0;
+  uint64_t timeout_ns = 2000000000ull;
+  int debug_skip_v_tile = -1;
+  bool profiling = false;
+  bool capturing = false;   // launches are being recorded into a unit program: no profiling events
+  EventPool ev_attn, ev_comb, ev_lat;
+  int last_split = 0, last_ctas = 0;
+  int64_t last_keys = 0;
+};
+
+namespace ws {
+
+// Entry-point bodies shared with the unit program (ws_api.cu).  Each validates
+// its arguments, updates the host bookkeeping and enqueues its launches on
+// `stream`; none synchronises.
+int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
+                cudaStream_t stream);
+int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
+                   const uint16_t* v_new, uint16_t* out, cudaStream_t stream);
+int flow_step_impl(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream);
+
+}  // namespace ws

@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "../../include/ws.h"
+#include "cache_state.cuh"
 #include "kernels.cuh"
 
 using namespace ws;
@@ -48,60 +49,6 @@ void ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced) {
   d.lanes = (n_qtiles + best_g - 1) / best_g;
   d.lane_ctas = best_cpl;
 }
-
-struct EventPool {
-  std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 end
-  int used = 0;
-  int64_t launches = 0;
-  double ms = 0.0;
-  void create(int pairs) {
-    ev.resize(2 * pairs);
-    for (auto& e : ev) cudaEventCreate(&e);
-    used = 0;
-  }
-  void destroy() {
-    for (auto& e : ev) cudaEventDestroy(e);
-    ev.clear();
-  }
-  void flush() {
-    for (int i = 0; i < used; ++i) {
-      cudaEventSynchronize(ev[2 * i + 1]);
-      float t = 0.f;
-      if (cudaEventElapsedTime(&t, ev[2 * i], ev[2 * i + 1]) == cudaSuccess) ms += t;
-    }
-    launches += used;
-    used = 0;
-  }
-  cudaEvent_t* next() {
-    if (ev.empty()) return nullptr;
-    if (2 * used >= (int)ev.size()) flush();
-    return &ev[2 * (used++)];
-  }
-};
-
-struct ws_cache {
-  ws_cache_config cfg{};
-  int device = 0;
-  int C = 0, T = 0, Nq = 0;
-  int64_t newest = -1;
-  std::vector<int64_t> slot_unit;     // C
-  std::vector<uint8_t> latent_ready;  // C * L
-  uint16_t* kv = nullptr;
-  size_t kv_bytes = 0;
-  float* part_o = nullptr;
-  float* part_ml = nullptr;
-  size_t ws_bytes = 0;
-  int* d_status = nullptr;
-  CUtensorMap kv_map;
-  int force_lane_ctas = 0;
-  int64_t slot_cap = 0;
-  uint64_t timeout_ns = 2000000000ull;
-  int debug_skip_v_tile = -1;
-  bool profiling = false;
-  EventPool ev_attn, ev_comb, ev_lat;
-  int last_split = 0, last_ctas = 0;
-  int64_t last_keys = 0;
-};
 
 namespace {
 
@@ -172,13 +119,13 @@ void free_all(ws_cache* h) {
 
 }  // namespace
 
-namespace {
+namespace ws {
 
 // Attention of the query units u_first .. u_first+n-1 at `layer` (one unit for
 // the per-unit step, several for a prefill).  Writes each unit's k_new/v_new
 // into its latent rows, plans each unit's visible runs, launches the kernel
 // and, when a head's key range was cut between CTAs, the merge.
-int attention_impl(ws_cache_t* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
+int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
                    const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
   if (!h || layer < 0 || layer >= h->cfg.n_layers || u_first < 0 || n < 1) return WS_ERR_ARG;
   if (n > kMaxQUnits) return WS_ERR_UNSUPPORTED;
@@ -258,7 +205,7 @@ int attention_impl(ws_cache_t* h, int layer, int64_t u_first, int n, const uint1
     a.head_dim = D;
     a.plane_rows = (int64_t)h->C * h->T;
     a.row0 = (int64_t)slot * h->T + h->cfg.n_cond;
-    cudaEvent_t* ev = h->profiling ? h->ev_lat.next() : nullptr;
+    cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_lat.next() : nullptr;
     if (ev) cudaEventRecord(ev[0], stream);
     if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
     if (ev) cudaEventRecord(ev[1], stream);
@@ -276,13 +223,13 @@ int attention_impl(ws_cache_t* h, int layer, int64_t u_first, int n, const uint1
   p.status = h->d_status;
   p.timeout_ns = h->timeout_ns;
   p.debug_skip_v_tile = h->debug_skip_v_tile;
-  cudaEvent_t* ev = h->profiling ? h->ev_attn.next() : nullptr;
+  cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_attn.next() : nullptr;
   if (ev) cudaEventRecord(ev[0], stream);
   int ctas = 0;
   if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
   if (any_split) {
-    ev = h->profiling ? h->ev_comb.next() : nullptr;
+    ev = h->profiling && !h->capturing ? h->ev_comb.next() : nullptr;
     if (ev) cudaEventRecord(ev[0], stream);
     if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
     if (ev) cudaEventRecord(ev[1], stream);
@@ -293,7 +240,57 @@ int attention_impl(ws_cache_t* h, int layer, int64_t u_first, int n, const uint1
   return WS_OK;
 }
 
-}  // namespace
+int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
+                cudaStream_t stream) {
+  if (!h || unit < 0 || (seg != WS_SEG_COND && seg != WS_SEG_LATENT)) return WS_ERR_ARG;
+  const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
+  if (n > 0) {
+    if (!k_slice || !v_slice) return WS_ERR_ARG;
+    if (!aligned16(k_slice) || !aligned16(v_slice)) return WS_ERR_ALIGN;
+  }
+  const size_t slot = (size_t)(unit % h->C);
+  if (seg == WS_SEG_COND) {
+    if (unit < h->newest) return WS_ERR_UNIT_ORDER;
+  } else {
+    const int st = resident(h, unit);
+    if (st != WS_OK) return st;
+  }
+  AppendParams p{};
+  p.src_k = k_slice;
+  p.src_v = v_slice;
+  p.cache = h->kv;
+  p.n_layers = h->cfg.n_layers;
+  p.layer0 = 0;
+  p.n_tokens = n;
+  p.n_heads = h->cfg.n_heads;
+  p.head_dim = h->cfg.head_dim;
+  p.plane_rows = (int64_t)h->C * h->T;
+  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  const cudaError_t e = launch_append(p, stream);
+  if (e != cudaSuccess) return WS_ERR_CUDA;
+  if (seg == WS_SEG_COND) {
+    if (unit > h->newest) {
+      h->slot_unit[slot] = unit;
+      std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
+                h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 0);
+      h->newest = unit;
+    }
+  } else {
+    std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
+              h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 1);
+  }
+  return WS_OK;
+}
+
+int flow_step_impl(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {
+  if (n < 0) return WS_ERR_ARG;
+  if (n == 0) return WS_OK;
+  if (!x || !v) return WS_ERR_ARG;
+  if (!aligned16(x) || !aligned16(v)) return WS_ERR_ALIGN;
+  return cuda_status(launch_euler(x, v, dt, n, stream));
+}
+
+}  // namespace ws
 
 extern "C" {
 
@@ -379,44 +376,7 @@ int ws_cache_destroy(ws_cache_t* h) {
 
 int ws_cache_append(ws_cache_t* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
                     cudaStream_t stream) {
-  if (!h || unit < 0 || (seg != WS_SEG_COND && seg != WS_SEG_LATENT)) return WS_ERR_ARG;
-  const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
-  if (n > 0) {
-    if (!k_slice || !v_slice) return WS_ERR_ARG;
-    if (!aligned16(k_slice) || !aligned16(v_slice)) return WS_ERR_ALIGN;
-  }
-  const size_t slot = (size_t)(unit % h->C);
-  if (seg == WS_SEG_COND) {
-    if (unit < h->newest) return WS_ERR_UNIT_ORDER;
-  } else {
-    const int st = resident(h, unit);
-    if (st != WS_OK) return st;
-  }
-  AppendParams p{};
-  p.src_k = k_slice;
-  p.src_v = v_slice;
-  p.cache = h->kv;
-  p.n_layers = h->cfg.n_layers;
-  p.layer0 = 0;
-  p.n_tokens = n;
-  p.n_heads = h->cfg.n_heads;
-  p.head_dim = h->cfg.head_dim;
-  p.plane_rows = (int64_t)h->C * h->T;
-  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
-  const cudaError_t e = launch_append(p, stream);
-  if (e != cudaSuccess) return WS_ERR_CUDA;
-  if (seg == WS_SEG_COND) {
-    if (unit > h->newest) {
-      h->slot_unit[slot] = unit;
-      std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
-                h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 0);
-      h->newest = unit;
-    }
-  } else {
-    std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
-              h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 1);
-  }
-  return WS_OK;
+  return append_impl(h, unit, seg, k_slice, v_slice, stream);
 }
 
 int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q, const uint16_t* k_new,
@@ -430,11 +390,7 @@ int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n
 }
 
 int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {
-  if (n < 0) return WS_ERR_ARG;
-  if (n == 0) return WS_OK;
-  if (!x || !v) return WS_ERR_ARG;
-  if (!aligned16(x) || !aligned16(v)) return WS_ERR_ALIGN;
-  return cuda_status(launch_euler(x, v, dt, n, stream));
+  return flow_step_impl(x, v, dt, n, stream);
 }
 
 int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg, uint16_t* k_out, uint16_t* v_out,

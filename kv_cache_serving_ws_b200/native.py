@@ -52,6 +52,18 @@ class ws_profile(C.Structure):
                 ("last_n_split", C.c_int32), ("last_ctas", C.c_int32), ("last_keys", C.c_int64)]
 
 
+class ws_unit_io(C.Structure):
+    _fields_ = [("n_steps", C.c_int32), ("out_per_call", C.c_int32), ("dt", C.c_float), ("n_latent", C.c_int64),
+                ("cond_k", C.c_void_p), ("cond_v", C.c_void_p), ("q", C.c_void_p), ("k_new", C.c_void_p),
+                ("v_new", C.c_void_p), ("out", C.c_void_p), ("x", C.c_void_p), ("vel", C.c_void_p),
+                ("commit_k", C.c_void_p), ("commit_v", C.c_void_p)]
+
+
+class ws_unit_graph_stats(C.Structure):
+    _fields_ = [("launches", C.c_int64), ("instantiations", C.c_int64), ("updates", C.c_int64),
+                ("nodes", C.c_int64), ("record_ms", C.c_double)]
+
+
 class WsError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -84,6 +96,10 @@ def _declare(lib):
                                       i64, C.POINTER(i32), C.POINTER(i32), i32, C.POINTER(i32)]),
         "ws_attention_noalloc": (C.c_int, [_P, _P, _P, i32, i32, i32, i32, _P]),
         "ws_debug_inject_stall": (C.c_int, [_P, C.c_int]),
+        "ws_unit_graph_create": (C.c_int, [C.POINTER(_P), _P, C.POINTER(ws_unit_io)]),
+        "ws_unit_graph_launch": (C.c_int, [_P, i64, _P]),
+        "ws_unit_graph_get_stats": (C.c_int, [_P, C.POINTER(ws_unit_graph_stats)]),
+        "ws_unit_graph_destroy": (C.c_int, [_P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -256,6 +272,32 @@ def ws_attention_noalloc(q, kv, out, n_query, n_keys, n_heads, head_dim, stream=
     """Attention over caller-owned K/V planes kv [2][H][Nk][D]; no device allocation."""
     return _done(lib().ws_attention_noalloc(_ptr(q), _ptr(kv), _ptr(out), n_query, n_keys, n_heads, head_dim,
                                             _stream(stream)), "ws_attention_noalloc", check)
+
+
+def ws_unit_graph_create(h, n_steps, dt, cond_k, cond_v, q, k_new, v_new, out, x, vel, commit_k, commit_v,
+                         out_per_call=True, n_latent=None, check=True):
+    """Unit program over cache h; the tensors must stay alive (and in place) while it exists."""
+    io = ws_unit_io(int(n_steps), 1 if out_per_call else 0, float(dt), int(x.numel() if n_latent is None else n_latent),
+                    _ptr(cond_k), _ptr(cond_v), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(x), _ptr(vel),
+                    _ptr(commit_k), _ptr(commit_v))
+    g = _P()
+    st = lib().ws_unit_graph_create(C.byref(g), h, C.byref(io))
+    _done(st, "ws_unit_graph_create", check)
+    return st, g
+
+
+def ws_unit_graph_launch(g, unit, stream=None, check=True):
+    return _done(lib().ws_unit_graph_launch(g, int(unit), _stream(stream)), "ws_unit_graph_launch", check)
+
+
+def ws_unit_graph_get_stats(g) -> dict:
+    st = ws_unit_graph_stats()
+    _done(lib().ws_unit_graph_get_stats(g, C.byref(st)), "ws_unit_graph_get_stats", True)
+    return {k: getattr(st, k) for k, _ in ws_unit_graph_stats._fields_}
+
+
+def ws_unit_graph_destroy(g, check=True):
+    return _done(lib().ws_unit_graph_destroy(g), "ws_unit_graph_destroy", check)
 
 
 def synth_fill(dst, key: int, index0: int = 0, stream=None):

@@ -57,7 +57,10 @@ V02 = Workload("v02-640x368-hist32-40x128", 1, 40, 128, 920, 4, 32, 32, seed=3, 
 RING = Workload("v02-640x368-ring128-u1000-40x128", 1, 40, 128, 920, 4, 32, 128, seed=4, unit=1000)
 FULL = Workload("v02-640x368-unit-40L-4steps-hist64-40x128", 40, 40, 128, 920, 4, 32, 64, seed=5, unit=64,
                 steps=4)
-ALL = {w.name: w for w in (TINY, V01, V02, RING, FULL)}
+# the same unit with a 32-unit history: the window one B200 can run inside the 160 ms unit
+FULL32 = Workload("v02-640x368-unit-40L-4steps-hist32-40x128", 40, 40, 128, 920, 4, 32, 32, seed=7, unit=32,
+                  steps=4)
+ALL = {w.name: w for w in (TINY, V01, V02, RING, FULL, FULL32)}
 
 
 def key(w: Workload, kind: int, unit: int = 0, layer: int = 0, step: int = 0) -> int:
