@@ -30,6 +30,13 @@ What each part follows:
   later one [remio 为什么端到端…].  Within the visible set the operation is the
   plain definition of softmax attention with scale 1/sqrt(D): s_j = q.k_j/sqrt(D),
   p_j = exp(s_j - max s) / sum exp(s - max s), out = sum_j p_j v_j.
+* Multi-unit queries (``UnitCache.prefill_attention``): several consecutive
+  query units at once, each over its own window, the same block-causal rule
+  [remio 为什么端到端…].
+* Sessions (``SessionPool``): independent conversations, one UnitCache each,
+  batched into one call; every query unit sees its own session only.  How many
+  conversations one deployment carries is the question the pages leave open
+  [remio 决定 Wan-Streamer 是否重要的三个信号].
 * Euler (``euler_step``): one flow-matching update x <- x + dt*v of the
   latent [rainbus 核心方法 (flow-matching latent generation)], evaluated as
   RN_bf16(fl64(x + fl64(dt*v))); dt*v is exact in fp64.
@@ -38,7 +45,8 @@ Parity pins (tests/test_oracle_*.py): brute-force full-sequence masked attention
 on tiny inputs, R-way splits of rows and heads (bit-identical), softmax row sums,
 closed forms (q = 0, constant V, one key, equal keys, two keys with logit gap ln 3),
 a torch float64 SDPA witness, exact-rational rounding for the bf16 conversion and
-the Euler step, and the ring's closed form.
+the Euler step, the ring's closed form, per-query-unit brute force for multi-unit
+queries, and per-session brute force plus session isolation for batched sessions.
 """
 from __future__ import annotations
 
@@ -341,6 +349,81 @@ class UnitCache:
             k, v, _ = self.visible_kv(layer, unit_first + j)
             outs.append(attention_rows(bf16_to_f64(q_bits[j]), k, v, rows=rows, heads=heads))
         return OK, np.stack(outs)
+
+
+class SessionPool:
+    """Several independent conversations served together (session economics:
+    remio.ai, section 决定 Wan-Streamer 是否重要的三个信号).  Each session is
+    its own UnitCache; one batched attention call takes query units of several
+    sessions, and each sees its own session's window only.
+
+    Query unit j of a call is (sessions[j], units[j]).  The units of one session
+    form a single stretch of consecutive units in the list, ending at that
+    session's newest unit; each stretch follows that session's prefill rules.
+    The list is checked stretch by stretch in order, and the first failing rule
+    gives the status.
+    """
+
+    def __init__(self, cfg: Config, n_sessions: int):
+        self.cfg = cfg
+        self.sessions = [UnitCache(cfg) for _ in range(n_sessions)]
+
+    def reset(self, session: int) -> int:
+        """The session's conversation ends; its ring starts empty."""
+        if not 0 <= session < len(self.sessions):
+            return ERR_ARG
+        self.sessions[session] = UnitCache(self.cfg)
+        return OK
+
+    def session_attention(self, layer: int, sessions, units, q_bits, k_new_bits, v_new_bits,
+                          rows=None, heads=None):
+        """Returns (status, out [n, rows, heads, D] float64)."""
+        c = self.cfg
+        n = len(sessions)
+        if not (0 <= layer < c.n_layers) or n < 1 or len(units) != n:
+            return ERR_ARG, None
+        if n > MAX_QUERY_UNITS:
+            return ERR_UNSUPPORTED, None
+        shape = (n, c.n_query, c.n_heads, c.head_dim)
+        if any(np.shape(a) != shape for a in (q_bits, k_new_bits, v_new_bits)):
+            return ERR_ARG, None
+        if any(not 0 <= s < len(self.sessions) for s in sessions) or any(u < 0 for u in units):
+            return ERR_ARG, None
+        stretches, seen, j = [], set(), 0
+        while j < n:
+            s = sessions[j]
+            if s in seen:
+                return ERR_ARG, None
+            seen.add(s)
+            k = j
+            while k + 1 < n and sessions[k + 1] == s:
+                if units[k + 1] != units[k] + 1:
+                    return ERR_ARG, None
+                k += 1
+            cache = self.sessions[s]
+            u_first, u_last = units[j], units[k]
+            if u_last > cache.newest:
+                return ERR_NOT_READY, None
+            if u_last < cache.newest:
+                return ERR_UNIT_ORDER, None
+            for u in range(u_first, u_last + 1):
+                st = cache._resident(u)
+                if st != OK:
+                    return st, None
+            for u in range(max(0, u_first - c.history_units), u_first):
+                if cache.slot_unit[cache.slot(u)] > u:
+                    return ERR_EVICTED, None
+            stretches.append((s, j, k))
+            j = k + 1
+        out = [None] * n
+        for s, j, k in stretches:
+            st, o = self.sessions[s].prefill_attention(layer, units[j], k - j + 1, q_bits[j:k + 1],
+                                                       k_new_bits[j:k + 1], v_new_bits[j:k + 1],
+                                                       rows=rows, heads=heads)
+            assert st == OK
+            for i in range(k - j + 1):
+                out[j + i] = o[i]
+        return OK, np.stack(out)
 
 
 def attention_flops(n_query: int, n_keys: int, n_heads: int, head_dim: int) -> float:

@@ -360,3 +360,103 @@ def test_prefill_error_rules():
     assert cache.prefill_attention(0, 3, 2, qs(2), qs(2), qs(2))[0] == orc.ERR_EVICTED   # 0 in unit 3's window
     assert cache.prefill_attention(0, 4, 1, qs(1), qs(1), qs(1))[0] == orc.OK            # window 1..4
     assert cache.prefill_attention(0, 0, 5, qs(5), qs(5), qs(5))[0] == orc.ERR_EVICTED   # query unit 0 gone
+
+
+# ------------------------------------------------------------- sessions --
+
+def _session_seq(cfg, seed, units, layer, current=None):
+    """Token sequence of one session for the brute force: committed units, and the
+    query units' latent rows from `current` = {unit: (k_new, v_new)}."""
+    seq = []
+    for uu in units:
+        cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+        ck = orc.bf16_to_f64(_bits(seed, synth.KIND_COND_K, cs, uu))[layer]
+        cv = orc.bf16_to_f64(_bits(seed, synth.KIND_COND_V, cs, uu))[layer]
+        seq += [(uu, "cond", ck[t], cv[t]) for t in range(cfg.n_cond)]
+        if current and uu in current:
+            lk, lv = (orc.bf16_to_f64(a) for a in current[uu])
+        else:
+            ls = (cfg.n_layers, cfg.n_query, cfg.n_heads, cfg.head_dim)
+            lk = orc.bf16_to_f64(_bits(seed, synth.KIND_COMMIT_K, ls, uu))[layer]
+            lv = orc.bf16_to_f64(_bits(seed, synth.KIND_COMMIT_V, ls, uu))[layer]
+        seq += [(uu, "latent", lk[t], lv[t]) for t in range(cfg.n_query)]
+    return seq
+
+
+def test_sessions_each_see_only_their_own_window():
+    """Three sessions at different points of their streams, batched in one call
+    (one streaming unit, one two-unit prefill, one streaming unit after a ring
+    wrap): every query unit equals the brute force over its own session's tokens."""
+    cfg = _cfg(history_units=2)                                  # C = 3
+    pool = orc.SessionPool(cfg, 4)
+    seeds = {0: 11, 1: 12, 2: 13}
+    hist = {0: list(range(0, 7)), 1: [0], 2: [40, 41]}           # session 0 wrapped twice
+    for s, units in hist.items():
+        _fill(pool.sessions[s], cfg, units, seed=seeds[s])
+    cs = (cfg.n_layers, cfg.n_cond, cfg.n_heads, cfg.head_dim)
+    assert pool.sessions[1].append(1, orc.SEG_COND, _bits(12, synth.KIND_COND_K, cs, 1),
+                                   _bits(12, synth.KIND_COND_V, cs, 1)) == orc.OK
+    sessions, units = [2, 1, 1, 0], [41, 0, 1, 6]
+    layer = 1
+    qs = (4, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q, kn, vn = (_bits(9, kind, qs, 0, layer) for kind in (synth.KIND_Q, synth.KIND_K_NEW, synth.KIND_V_NEW))
+    st, out = pool.session_attention(layer, sessions, units, q, kn, vn)
+    assert st == orc.OK and out.shape == (4, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    for s in (0, 1, 2):
+        js = [j for j in range(4) if sessions[j] == s]
+        mine = {units[j]: (kn[j], vn[j]) for j in js}
+        every = sorted(set(hist[s]) | set(mine))
+        seq = _session_seq(cfg, seeds[s], every, layer, current=mine)
+        for j in js:
+            want = _brute_force(cfg, seq, units[j], layer, orc.bf16_to_f64(q[j]))
+            assert np.max(np.abs(out[j] - want)) <= 1e-12, (s, units[j])
+    # session 3 was never touched; the others' bookkeeping is their own
+    assert pool.sessions[3].slot_table() == [-1, -1, -1]
+    assert pool.sessions[0].slot_table() == [6, 4, 5]
+    assert pool.sessions[2].slot_table() == [-1, 40, 41]
+
+
+def test_sessions_batch_equals_separate_calls_bit_for_bit():
+    """Routing pin: the batched call gives exactly what each session's own call gives
+    (rows are independent in the definition)."""
+    cfg = _cfg(history_units=3)
+    a, b = orc.SessionPool(cfg, 3), orc.SessionPool(cfg, 3)
+    for pool in (a, b):
+        for s in range(3):
+            _fill(pool.sessions[s], cfg, list(range(s, s + 4 + s)), seed=20 + s)
+    units = [s + 3 + s for s in range(3)]
+    qs = (3, cfg.n_query, cfg.n_heads, cfg.head_dim)
+    q, kn, vn = (_bits(5, kind, qs) for kind in (synth.KIND_Q, synth.KIND_K_NEW, synth.KIND_V_NEW))
+    st, out = a.session_attention(0, [0, 1, 2], units, q, kn, vn)
+    assert st == orc.OK
+    for s in range(3):
+        st1, o1 = b.sessions[s].unit_attention(0, units[s], q[s], kn[s], vn[s])
+        assert st1 == orc.OK and np.array_equal(o1, out[s])
+
+
+def test_session_error_rules_and_reset():
+    cfg = _cfg(history_units=3)                                  # C = 4
+    pool = orc.SessionPool(cfg, 3)
+    _fill(pool.sessions[0], cfg, [0, 1, 2], commit=False)
+    _fill(pool.sessions[1], cfg, [5], commit=False)
+    z = lambda n: np.zeros((n, cfg.n_query, cfg.n_heads, cfg.head_dim), np.uint16)
+    call = lambda ss, uu: pool.session_attention(0, ss, uu, z(len(ss)), z(len(ss)), z(len(ss)))[0]
+    assert call([0, 1], [2, 5]) == orc.OK
+    assert call([1, 0], [5, 2]) == orc.OK                        # any session order
+    assert call([0, 1, 0], [2, 5, 2]) == orc.ERR_ARG             # a session in two stretches
+    assert call([0, 0], [1, 1]) == orc.ERR_ARG                   # same unit twice
+    assert call([0, 0], [0, 2]) == orc.ERR_ARG                   # not consecutive
+    assert call([0, 3], [2, 0]) == orc.ERR_ARG                   # no such session
+    assert call([0, 1], [2, -1]) == orc.ERR_ARG
+    assert call([0, 2], [2, 0]) == orc.ERR_NOT_READY             # session 2 empty
+    assert call([1, 0], [5, 1]) == orc.ERR_UNIT_ORDER            # session 0's newest is 2
+    assert call([0, 0, 0], [0, 1, 2]) == orc.OK                  # a prefill stretch
+    assert call([2, 0], [0, 1]) == orc.ERR_NOT_READY             # first failing stretch decides
+    assert call([0] * 65, list(range(65))) == orc.ERR_UNSUPPORTED
+    _fill(pool.sessions[0], cfg, [3, 4], commit=False)           # unit 4 takes unit 0's slot
+    assert call([0, 0, 0, 0], [1, 2, 3, 4]) == orc.ERR_EVICTED
+    assert pool.reset(0) == orc.OK and pool.reset(3) == orc.ERR_ARG
+    assert pool.sessions[0].slot_table() == [-1] * 4
+    assert call([0], [4]) == orc.ERR_NOT_READY
+    _fill(pool.sessions[0], cfg, [100], commit=False)            # a new conversation at any unit index
+    assert call([0, 1], [100, 5]) == orc.OK
