@@ -712,6 +712,82 @@ def run_schedule(args):
             sys.exit(1)
 
 
+def run_sessions(args):
+    """Concurrent sessions: N conversations in one pool, their current units in one
+    attention launch, against N separate launches (one layer, steady-state windows).
+    Two stream shapes: the 640x368 stream with a 32-unit history and the 192x336
+    stream with a 16-unit history."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200 import synth
+    from kv_cache_serving_ws_b200.workloads import V01, V02
+    for w, n in ((V02, args.sessions), (V01, 4 * args.sessions)):
+        n = min(n, 64)
+        _, h = ws.ws_pool_create(ws.make_config(1, w.n_heads, w.head_dim, w.n_video, w.n_audio, w.n_cond,
+                                                w.history_units), n)
+        dev = torch.device("cuda")
+        bf = torch.bfloat16
+        ck = torch.empty((1, w.n_cond, w.n_heads, w.head_dim), dtype=bf, device=dev)
+        cv = torch.empty_like(ck)
+        lk = torch.empty((1, w.n_query, w.n_heads, w.head_dim), dtype=bf, device=dev)
+        lv = torch.empty_like(lk)
+        units = []
+        for s in range(n):
+            first = 7 * s                                   # sessions at different stream positions
+            for u in range(first, first + w.history_units + 1):
+                ws.synth_fill(ck, synth.stream_key(w.seed + 1000 * s, synth.KIND_COND_K, u))
+                ws.synth_fill(cv, synth.stream_key(w.seed + 1000 * s, synth.KIND_COND_V, u))
+                ws.ws_session_append(h, s, u, ws.WS_SEG_COND, ck, cv)
+                if u < first + w.history_units:
+                    ws.synth_fill(lk, synth.stream_key(w.seed + 1000 * s, synth.KIND_COMMIT_K, u))
+                    ws.synth_fill(lv, synth.stream_key(w.seed + 1000 * s, synth.KIND_COMMIT_V, u))
+                    ws.ws_session_append(h, s, u, ws.WS_SEG_LATENT, lk, lv)
+            units.append(first + w.history_units)
+        shape = (n, w.n_query, w.n_heads, w.head_dim)
+        q = torch.empty(shape, dtype=bf, device=dev)
+        kn, vn, out = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+        ws.synth_fill(q, synth.stream_key(w.seed, synth.KIND_Q, 0))
+        ws.synth_fill(kn, synth.stream_key(w.seed, synth.KIND_K_NEW, 0))
+        ws.synth_fill(vn, synth.stream_key(w.seed, synth.KIND_V_NEW, 0))
+        sess = list(range(n))
+
+        def batched():
+            ws.ws_session_attention(h, 0, sess, units, q, kn, vn, out)
+
+        def separate():
+            for s in sess:
+                ws.ws_session_attention(h, 0, [s], [units[s]], q[s], kn[s], vn[s], out[s])
+
+        def timed(fn):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(args.calls):
+                fn()
+            e1.record()
+            torch.cuda.synchronize()
+            return e0.elapsed_time(e1) / args.calls
+
+        ms_b = timed(batched)
+        ms_s = timed(separate)
+        st = ws.ws_sync(h, check=False)
+        flops = n * w.flops_per_call()
+        print(json.dumps({"mode": "sessions", "workload": w.name, "sessions": n, "keys_per_query": w.n_keys,
+                          "batched": {"ms_per_call": round(ms_b, 4), "TFLOP/s": round(flops / ms_b / 1e9, 1),
+                                      "attention_launches": 1},
+                          "separate": {"ms_per_call": round(ms_s, 4), "TFLOP/s": round(flops / ms_s / 1e9, 1),
+                                       "attention_launches": n},
+                          "speedup": round(ms_s / ms_b, 3), "status": ws.status_string(st)}), flush=True)
+        ws.ws_cache_destroy(h)
+        del q, kn, vn, out
+        torch.cuda.empty_cache()
+        if st != ws.WS_OK:
+            sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -728,6 +804,8 @@ def main():
     ap.add_argument("--schedule", action="store_true",
                     help="per-unit schedule: direct calls vs the unit program, back to back and paced at 160 ms")
     ap.add_argument("--units", type=int, default=24)
+    ap.add_argument("--sessions", type=int, default=0,
+                    help="concurrent sessions: N conversations batched in one launch vs N launches")
     args = ap.parse_args()
     if args.case:
         run_case(args)
@@ -737,6 +815,9 @@ def main():
         return
     if args.schedule:
         run_schedule(args)
+        return
+    if args.sessions:
+        run_sessions(args)
         return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

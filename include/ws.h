@@ -193,6 +193,7 @@ typedef struct {
   int64_t newest_unit;         /* -1 before the first append */
   uint64_t cache_bytes;        /* K and V planes */
   uint64_t workspace_bytes;    /* split-K partials */
+  int32_t n_sessions;          /* 1 for ws_cache_create */
 } ws_cache_info;
 
 int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info);
@@ -334,6 +335,7 @@ typedef struct {
   const uint16_t* vel;
   const uint16_t* commit_k;
   const uint16_t* commit_v;
+  int32_t session;              /* session of a pool (0 for a plain cache) */
 } ws_unit_io;
 
 typedef struct ws_unit_graph ws_unit_graph_t;   /* opaque */
@@ -372,6 +374,58 @@ int ws_unit_graph_get_stats(const ws_unit_graph_t* g, ws_unit_graph_stats* out);
 
 /* Destroy a program (synchronises its pending launches first). */
 int ws_unit_graph_destroy(ws_unit_graph_t* g);
+
+/*
+ * Concurrent sessions -- several independent conversations, each with its own
+ * unit ring, served by one cache (a pool) and batched into single attention
+ * launches.  How many concurrent conversations one deployment can carry is the
+ * open question of session economics (remio.ai, section
+ * 决定 Wan-Streamer 是否重要的三个信号).
+ *
+ * ws_pool_create -- a cache of n_sessions rings of C = U+1 slots each, in one
+ * allocation: K and V planes [L][2][H][n_sessions*C*T][D] bf16, session s owning
+ * rows [s*C*T, (s+1)*C*T) of each plane.  Every session starts empty.  The
+ * single-session entry points (ws_cache_append, ws_unit_attention,
+ * ws_prefill_attention, ws_cache_read, ws_cache_slot_table) address session 0;
+ * ws_cache_create(cfg) is ws_pool_create(cfg, 1).
+ * Errors: as ws_cache_create; WS_ERR_ARG for n_sessions < 1;
+ * WS_ERR_UNSUPPORTED when n_sessions*C*T >= 2^31.
+ */
+int ws_pool_create(ws_cache_t** out, const ws_cache_config* cfg, int32_t n_sessions, cudaStream_t stream);
+
+/* ws_cache_append / ws_cache_read / ws_cache_slot_table on one session of a pool
+ * (same contracts; WS_ERR_ARG for a session outside [0, n_sessions)). */
+int ws_session_append(ws_cache_t* h, int32_t session, int64_t unit, int seg,
+                      const uint16_t* k_slice, const uint16_t* v_slice, cudaStream_t stream);
+int ws_session_read(ws_cache_t* h, int32_t session, int layer, int64_t unit, int seg,
+                    uint16_t* k_out, uint16_t* v_out, cudaStream_t stream);
+int ws_session_slot_table(const ws_cache_t* h, int32_t session, int64_t* slot_unit_host);
+
+/* A conversation ends: its session's ring is emptied (every slot free, no
+ * newest unit), so a new conversation can start in it at any unit index.  Host
+ * bookkeeping only; work already enqueued is unaffected. */
+int ws_session_reset(ws_cache_t* h, int32_t session);
+
+/*
+ * ws_session_attention -- one launch of block-causal attention for n query
+ * units of several sessions: query unit j is unit units[j] of session
+ * sessions[j] (host arrays), with its queries, current-unit K/V and output at
+ * rows [j*Nq, (j+1)*Nq) of q, k_new, v_new, out ([n][Nq][H][D] bf16).  Each
+ * query unit writes its k_new/v_new into its session's slot and attends over
+ * its own session's window only, exactly as ws_unit_attention on that session
+ * would.  The units of one session form one stretch of consecutive units in
+ * the list (one unit for a streaming step, several for a prefill), the last of
+ * which is that session's newest unit.  1 <= n <= 64.
+ * Errors: WS_ERR_ARG (a session outside the pool, a session in two stretches
+ * or a stretch of non-consecutive units, NULL, negative unit),
+ * WS_ERR_ALIGN, WS_ERR_NOT_READY / WS_ERR_UNIT_ORDER / WS_ERR_EVICTED per
+ * session as for ws_prefill_attention, WS_ERR_UNSUPPORTED (n > 64, or more
+ * visible row runs than one launch holds), WS_ERR_CUDA.  On an error nothing
+ * is launched or recorded.
+ */
+int ws_session_attention(ws_cache_t* h, int layer, int32_t n, const int32_t* sessions,
+                         const int64_t* units, const uint16_t* q, const uint16_t* k_new,
+                         const uint16_t* v_new, uint16_t* out, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

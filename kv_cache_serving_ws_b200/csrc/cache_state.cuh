@@ -41,13 +41,23 @@ struct EventPool {
   }
 };
 
+// Ring bookkeeping of one session (one conversation's stream of units).
+struct Ring {
+  int64_t newest = -1;
+  std::vector<int64_t> slot_unit;     // C entries, -1 = empty
+  std::vector<uint8_t> latent_ready;  // C * L: slot s holds latent rows of layer l
+};
+
+// A cache holds n_sessions independent rings in one allocation: session s owns
+// rows [s*C*T, (s+1)*C*T) of every (layer, K|V, head) plane, so one tensor map
+// covers every session and one attention launch can serve several of them.
 struct ws_cache {
   ws_cache_config cfg{};
   int device = 0;
   int C = 0, T = 0, Nq = 0;
-  int64_t newest = -1;
-  std::vector<int64_t> slot_unit;     // C
-  std::vector<uint8_t> latent_ready;  // C * L
+  int n_sessions = 1;
+  int64_t session_rows = 0;           // C * T
+  std::vector<Ring> rings;            // one per session
   uint16_t* kv = nullptr;
   size_t kv_bytes = 0;
   float* part_o = nullptr;
@@ -71,10 +81,12 @@ namespace ws {
 // Entry-point bodies shared with the unit program (ws_api.cu).  Each validates
 // its arguments, updates the host bookkeeping and enqueues its launches on
 // `stream`; none synchronises.
-int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
+int append_impl(ws_cache* h, int session, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
                 cudaStream_t stream);
-int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
-                   const uint16_t* v_new, uint16_t* out, cudaStream_t stream);
+// Query unit j is (sessions[j], units[j]); its queries are rows [j*Nq, (j+1)*Nq)
+// of q, k_new, v_new and out.
+int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_t* units, int n, const uint16_t* q,
+                   const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream);
 int flow_step_impl(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream);
 
 }  // namespace ws

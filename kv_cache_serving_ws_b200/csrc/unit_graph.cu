@@ -35,20 +35,17 @@ namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Host bookkeeping of the cache, restored when recording a unit fails halfway.
+// Host bookkeeping of the program's session, restored when recording a unit fails halfway.
 struct Snapshot {
-  int64_t newest;
-  std::vector<int64_t> slot_unit;
-  std::vector<uint8_t> latent_ready;
+  int session;
+  Ring ring;
   int last_split, last_ctas;
   int64_t last_keys;
-  explicit Snapshot(const ws_cache* h)
-      : newest(h->newest), slot_unit(h->slot_unit), latent_ready(h->latent_ready), last_split(h->last_split),
-        last_ctas(h->last_ctas), last_keys(h->last_keys) {}
+  Snapshot(const ws_cache* h, int s)
+      : session(s), ring(h->rings[(size_t)s]), last_split(h->last_split), last_ctas(h->last_ctas),
+        last_keys(h->last_keys) {}
   void restore(ws_cache* h) const {
-    h->newest = newest;
-    h->slot_unit = slot_unit;
-    h->latent_ready = latent_ready;
+    h->rings[(size_t)session] = ring;
     h->last_split = last_split;
     h->last_ctas = last_ctas;
     h->last_keys = last_keys;
@@ -61,16 +58,17 @@ int record_unit(ws_unit_graph* g, int64_t unit, cudaStream_t s) {
   const ws_unit_io& io = g->io;
   const int L = h->cfg.n_layers;
   const size_t call_elems = (size_t)h->Nq * h->cfg.n_heads * h->cfg.head_dim;
-  int st = ws::append_impl(h, unit, WS_SEG_COND, io.cond_k, io.cond_v, s);
+  const int32_t sess = io.session;
+  int st = ws::append_impl(h, sess, unit, WS_SEG_COND, io.cond_k, io.cond_v, s);
   for (int step = 0; step < io.n_steps && st == WS_OK; ++step) {
     for (int l = 0; l < L && st == WS_OK; ++l) {
       const size_t off = ((size_t)step * L + l) * call_elems;
-      st = ws::attention_impl(h, l, unit, 1, io.q + off, io.k_new + off, io.v_new + off,
+      st = ws::attention_impl(h, l, &sess, &unit, 1, io.q + off, io.k_new + off, io.v_new + off,
                               io.out + (io.out_per_call ? off : 0), s);
     }
     if (st == WS_OK) st = ws::flow_step_impl(io.x, io.vel + (size_t)step * io.n_latent, io.dt, io.n_latent, s);
   }
-  if (st == WS_OK) st = ws::append_impl(h, unit, WS_SEG_LATENT, io.commit_k, io.commit_v, s);
+  if (st == WS_OK) st = ws::append_impl(h, sess, unit, WS_SEG_LATENT, io.commit_k, io.commit_v, s);
   return st;
 }
 
@@ -80,6 +78,7 @@ extern "C" {
 
 int ws_unit_graph_create(ws_unit_graph_t** out, ws_cache_t* h, const ws_unit_io* io) {
   if (!out || !h || !io || io->n_steps < 1 || io->n_latent < 0) return WS_ERR_ARG;
+  if (io->session < 0 || io->session >= h->n_sessions) return WS_ERR_ARG;
   const void* ptrs[] = {io->cond_k, io->cond_v, io->q, io->k_new, io->v_new, io->out,
                         io->x, io->vel, io->commit_k, io->commit_v};
   for (const void* p : ptrs) {
@@ -107,7 +106,7 @@ int ws_unit_graph_launch(ws_unit_graph_t* g, int64_t unit, cudaStream_t stream) 
   if (!g || unit < 0) return WS_ERR_ARG;
   ws_cache* h = g->h;
   const auto t0 = std::chrono::steady_clock::now();
-  const Snapshot before(h);
+  const Snapshot before(h, g->io.session);
 
   if (cudaStreamBeginCapture(g->cap, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
     cudaGetLastError();

@@ -68,10 +68,10 @@ bool config_ok(const ws_cache_config* c) {
   return true;
 }
 
-// status of `unit` in the ring: resident, evicted (its slot holds a newer unit) or never appended
-int resident(const ws_cache* h, int64_t unit) {
+// status of `unit` in a session's ring: resident, evicted (its slot holds a newer unit) or never appended
+int resident(const ws_cache* h, int session, int64_t unit) {
   if (unit < 0) return WS_ERR_ARG;
-  const int64_t holder = h->slot_unit[(size_t)(unit % h->C)];
+  const int64_t holder = h->rings[(size_t)session].slot_unit[(size_t)(unit % h->C)];
   if (holder == unit) return WS_OK;
   return holder > unit ? WS_ERR_EVICTED : WS_ERR_NOT_READY;
 }
@@ -121,33 +121,56 @@ void free_all(ws_cache* h) {
 
 namespace ws {
 
-// Attention of the query units u_first .. u_first+n-1 at `layer` (one unit for
-// the per-unit step, several for a prefill).  Writes each unit's k_new/v_new
-// into its latent rows, plans each unit's visible runs, launches the kernel
-// and, when a head's key range was cut between CTAs, the merge.
-int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_t* q, const uint16_t* k_new,
-                   const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
-  if (!h || layer < 0 || layer >= h->cfg.n_layers || u_first < 0 || n < 1) return WS_ERR_ARG;
+// Attention of n query units at `layer`: the current unit of several sessions,
+// and/or consecutive units of one session (a prefill).  Writes each unit's
+// k_new/v_new into its latent rows, plans each unit's visible runs in its
+// session's rows, launches the kernel and, when a head's key range was cut
+// between CTAs, the merge.
+int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_t* units, int n, const uint16_t* q,
+                   const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  if (!h || layer < 0 || layer >= h->cfg.n_layers || !sessions || !units || n < 1) return WS_ERR_ARG;
   if (n > kMaxQUnits) return WS_ERR_UNSUPPORTED;
   if (!q || !k_new || !v_new || !out) return WS_ERR_ARG;
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(out)) return WS_ERR_ALIGN;
-  const int64_t u_last = u_first + n - 1;
-  if (h->newest < 0 || u_last > h->newest) return WS_ERR_NOT_READY;
-  if (u_last < h->newest) return WS_ERR_UNIT_ORDER;
   const int H = h->cfg.n_heads, D = h->cfg.head_dim, L = h->cfg.n_layers, U = h->cfg.history_units;
-  // every query unit must be resident, and no unit of any query window evicted
-  for (int64_t u = u_first; u <= u_last; ++u) {
-    const int st = resident(h, u);
-    if (st != WS_OK) return st;
+  const int S = h->n_sessions;
+  for (int j = 0; j < n; ++j)
+    if (sessions[j] < 0 || sessions[j] >= S || units[j] < 0) return WS_ERR_ARG;
+  // The query units of one session form one stretch of consecutive units in the
+  // list, ending at the session's newest unit.  Every query unit must be
+  // resident, and no unit of any query window evicted.
+  std::vector<uint8_t> seen((size_t)S, 0);
+  for (int j = 0; j < n;) {
+    const int sess = sessions[j];
+    if (seen[(size_t)sess]) return WS_ERR_ARG;
+    seen[(size_t)sess] = 1;
+    int k = j;
+    while (k + 1 < n && sessions[k + 1] == sess) {
+      if (units[k + 1] != units[k] + 1) return WS_ERR_ARG;
+      ++k;
+    }
+    const Ring& r = h->rings[(size_t)sess];
+    const int64_t u_first = units[j], u_last = units[k];
+    if (r.newest < 0 || u_last > r.newest) return WS_ERR_NOT_READY;
+    if (u_last < r.newest) return WS_ERR_UNIT_ORDER;
+    for (int64_t u = u_first; u <= u_last; ++u) {
+      const int st = resident(h, sess, u);
+      if (st != WS_OK) return st;
+    }
+    // units before the first query unit lie in some query window; one whose slot
+    // now holds a newer unit (a later query unit of a long prefill) is gone
+    for (int64_t u = std::max<int64_t>(0, u_first - U); u < u_first; ++u)
+      if (r.slot_unit[(size_t)(u % h->C)] > u) return WS_ERR_EVICTED;
+    j = k + 1;
   }
-  // units before the first query unit lie in some query window; one whose slot
-  // now holds a newer unit (a later query unit of a long prefill) is gone
-  for (int64_t u = std::max<int64_t>(0, u_first - U); u < u_first; ++u)
-    if (h->slot_unit[(size_t)(u % h->C)] > u) return WS_ERR_EVICTED;
 
   // plan first (pure host work), so that an unsupported layout changes nothing
-  std::vector<uint8_t> ready(h->latent_ready);
-  for (int64_t u = u_first; u <= u_last; ++u) ready[(size_t)(u % h->C) * L + layer] = 1;
+  std::vector<std::vector<uint8_t>> ready((size_t)S);
+  for (int j = 0; j < n; ++j) {
+    auto& rd = ready[(size_t)sessions[j]];
+    if (rd.empty()) rd = h->rings[(size_t)sessions[j]].latent_ready;
+    rd[(size_t)(units[j] % h->C) * L + layer] = 1;
+  }
   AttnParams p{};
   p.qu.n_units = n;
   p.qu.rows = h->Nq;
@@ -157,11 +180,13 @@ int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_
     p.qu.run_first[j] = runs;
     p.qu.tile_start[j] = tiles;
     int32_t nr = 0;
-    const int st = plan_runs(h->cfg, h->slot_unit.data(), ready.data(), layer, u_first + j, p.runs.row_begin + runs,
-                             p.runs.rows + runs, kMaxRuns - runs, &nr);
+    const int sess = sessions[j];
+    const int st = plan_runs(h->cfg, h->rings[(size_t)sess].slot_unit.data(), ready[(size_t)sess].data(), layer,
+                             units[j], p.runs.row_begin + runs, p.runs.rows + runs, kMaxRuns - runs, &nr);
     if (st != WS_OK) return st;
     int t = 0;
     for (int r = runs; r < runs + nr; ++r) {
+      p.runs.row_begin[r] += (int32_t)(sess * h->session_rows);
       p.runs.tile_begin[r] = t;
       t += (p.runs.rows[r] + kBlockN - 1) / kBlockN;
       keys += p.runs.rows[r];
@@ -193,7 +218,7 @@ int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_
   // 1. the query units' latent K/V of this layer into their slots
   const size_t unit_elems = (size_t)h->Nq * H * D;
   for (int j = 0; j < n; ++j) {
-    const size_t slot = (size_t)((u_first + j) % h->C);
+    const size_t slot = (size_t)(units[j] % h->C);
     AppendParams a{};
     a.src_k = k_new + j * unit_elems;
     a.src_v = v_new + j * unit_elems;
@@ -203,13 +228,13 @@ int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_
     a.n_tokens = h->Nq;
     a.n_heads = H;
     a.head_dim = D;
-    a.plane_rows = (int64_t)h->C * h->T;
-    a.row0 = (int64_t)slot * h->T + h->cfg.n_cond;
+    a.plane_rows = h->session_rows * h->n_sessions;
+    a.row0 = sessions[j] * h->session_rows + (int64_t)slot * h->T + h->cfg.n_cond;
     cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_lat.next() : nullptr;
     if (ev) cudaEventRecord(ev[0], stream);
     if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
     if (ev) cudaEventRecord(ev[1], stream);
-    h->latent_ready[slot * L + layer] = 1;
+    h->rings[(size_t)sessions[j]].latent_ready[slot * L + layer] = 1;
   }
 
   // 2. attention (+ merge of the partials of cut items)
@@ -240,9 +265,11 @@ int attention_impl(ws_cache* h, int layer, int64_t u_first, int n, const uint16_
   return WS_OK;
 }
 
-int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
+int append_impl(ws_cache* h, int session, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
                 cudaStream_t stream) {
   if (!h || unit < 0 || (seg != WS_SEG_COND && seg != WS_SEG_LATENT)) return WS_ERR_ARG;
+  if (session < 0 || session >= h->n_sessions) return WS_ERR_ARG;
+  Ring& r = h->rings[(size_t)session];
   const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
   if (n > 0) {
     if (!k_slice || !v_slice) return WS_ERR_ARG;
@@ -250,9 +277,9 @@ int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, con
   }
   const size_t slot = (size_t)(unit % h->C);
   if (seg == WS_SEG_COND) {
-    if (unit < h->newest) return WS_ERR_UNIT_ORDER;
+    if (unit < r.newest) return WS_ERR_UNIT_ORDER;
   } else {
-    const int st = resident(h, unit);
+    const int st = resident(h, session, unit);
     if (st != WS_OK) return st;
   }
   AppendParams p{};
@@ -264,20 +291,20 @@ int append_impl(ws_cache* h, int64_t unit, int seg, const uint16_t* k_slice, con
   p.n_tokens = n;
   p.n_heads = h->cfg.n_heads;
   p.head_dim = h->cfg.head_dim;
-  p.plane_rows = (int64_t)h->C * h->T;
-  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  p.plane_rows = h->session_rows * h->n_sessions;
+  p.row0 = session * h->session_rows + (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
   const cudaError_t e = launch_append(p, stream);
   if (e != cudaSuccess) return WS_ERR_CUDA;
   if (seg == WS_SEG_COND) {
-    if (unit > h->newest) {
-      h->slot_unit[slot] = unit;
-      std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
-                h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 0);
-      h->newest = unit;
+    if (unit > r.newest) {
+      r.slot_unit[slot] = unit;
+      std::fill(r.latent_ready.begin() + slot * h->cfg.n_layers, r.latent_ready.begin() + (slot + 1) * h->cfg.n_layers,
+                0);
+      r.newest = unit;
     }
   } else {
-    std::fill(h->latent_ready.begin() + slot * h->cfg.n_layers,
-              h->latent_ready.begin() + (slot + 1) * h->cfg.n_layers, 1);
+    std::fill(r.latent_ready.begin() + slot * h->cfg.n_layers, r.latent_ready.begin() + (slot + 1) * h->cfg.n_layers,
+              1);
   }
   return WS_OK;
 }
@@ -318,9 +345,11 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit, const 
   return plan_runs(*cfg, slot_unit, latent_ready, layer, unit, row_begin, rows, max_runs, n_runs);
 }
 
-int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t stream) {
-  if (!out || !config_ok(cfg)) return WS_ERR_ARG;
+int ws_pool_create(ws_cache_t** out, const ws_cache_config* cfg, int32_t n_sessions, cudaStream_t stream) {
+  if (!out || !config_ok(cfg) || n_sessions < 1) return WS_ERR_ARG;
   if (cfg->head_dim != 64 && cfg->head_dim != 128) return WS_ERR_UNSUPPORTED;
+  const int64_t T64 = (int64_t)cfg->n_cond + cfg->n_video + cfg->n_audio;
+  if (T64 * (cfg->history_units + 1) * n_sessions >= (int64_t)1 << 31) return WS_ERR_UNSUPPORTED;
   ws_cache* h = new (std::nothrow) ws_cache();
   if (!h) return WS_ERR_OOM;
   h->cfg = *cfg;
@@ -328,14 +357,19 @@ int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t s
   h->Nq = cfg->n_video + cfg->n_audio;
   h->T = cfg->n_cond + h->Nq;
   h->C = cfg->history_units + 1;
-  h->slot_unit.assign(h->C, -1);
-  h->latent_ready.assign((size_t)h->C * cfg->n_layers, 0);
+  h->n_sessions = n_sessions;
+  h->session_rows = (int64_t)h->C * h->T;
+  h->rings.resize((size_t)n_sessions);
+  for (Ring& r : h->rings) {
+    r.slot_unit.assign(h->C, -1);
+    r.latent_ready.assign((size_t)h->C * cfg->n_layers, 0);
+  }
   if (const char* t = std::getenv("WS_WAIT_TIMEOUT_MS")) {
     const long long ms = std::atoll(t);
     if (ms > 0) h->timeout_ns = (uint64_t)ms * 1000000ull;
   }
   const int L = cfg->n_layers, H = cfg->n_heads, D = cfg->head_dim;
-  const int64_t rows = (int64_t)h->C * h->T;
+  const int64_t rows = h->session_rows * n_sessions;
   h->kv_bytes = (size_t)L * 2 * H * rows * D * 2;
   // partial slots: two per CTA; an automatic decomposition has at most one CTA
   // per SM (more only when the query blocks outnumber the SMs)
@@ -362,6 +396,10 @@ int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t s
   return WS_OK;
 }
 
+int ws_cache_create(ws_cache_t** out, const ws_cache_config* cfg, cudaStream_t stream) {
+  return ws_pool_create(out, cfg, 1, stream);
+}
+
 int ws_cache_destroy(ws_cache_t* h) {
   if (!h) return WS_OK;
   int dev = 0;
@@ -376,36 +414,58 @@ int ws_cache_destroy(ws_cache_t* h) {
 
 int ws_cache_append(ws_cache_t* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
                     cudaStream_t stream) {
-  return append_impl(h, unit, seg, k_slice, v_slice, stream);
+  return append_impl(h, 0, unit, seg, k_slice, v_slice, stream);
+}
+
+int ws_session_append(ws_cache_t* h, int32_t session, int64_t unit, int seg, const uint16_t* k_slice,
+                      const uint16_t* v_slice, cudaStream_t stream) {
+  return append_impl(h, session, unit, seg, k_slice, v_slice, stream);
 }
 
 int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q, const uint16_t* k_new,
                       const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
-  return attention_impl(h, layer, unit, 1, q, k_new, v_new, out, stream);
+  const int32_t s0 = 0;
+  return attention_impl(h, layer, &s0, &unit, 1, q, k_new, v_new, out, stream);
 }
 
 int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n_units, const uint16_t* q,
                          const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
-  return attention_impl(h, layer, unit_first, n_units, q, k_new, v_new, out, stream);
+  if (!h || unit_first < 0 || n_units < 1) return WS_ERR_ARG;
+  if (n_units > kMaxQUnits) return WS_ERR_UNSUPPORTED;
+  int32_t sess[kMaxQUnits];
+  int64_t units[kMaxQUnits];
+  for (int j = 0; j < n_units; ++j) {
+    sess[j] = 0;
+    units[j] = unit_first + j;
+  }
+  return attention_impl(h, layer, sess, units, n_units, q, k_new, v_new, out, stream);
+}
+
+int ws_session_attention(ws_cache_t* h, int layer, int32_t n, const int32_t* sessions, const int64_t* units,
+                         const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, uint16_t* out,
+                         cudaStream_t stream) {
+  return attention_impl(h, layer, sessions, units, n, q, k_new, v_new, out, stream);
 }
 
 int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {
   return flow_step_impl(x, v, dt, n, stream);
 }
 
-int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg, uint16_t* k_out, uint16_t* v_out,
-                  cudaStream_t stream) {
+int ws_session_read(ws_cache_t* h, int32_t session, int layer, int64_t unit, int seg, uint16_t* k_out,
+                    uint16_t* v_out, cudaStream_t stream) {
   if (!h || layer < 0 || layer >= h->cfg.n_layers || unit < 0) return WS_ERR_ARG;
+  if (session < 0 || session >= h->n_sessions) return WS_ERR_ARG;
   if (seg != WS_SEG_COND && seg != WS_SEG_LATENT) return WS_ERR_ARG;
   const int n = seg == WS_SEG_COND ? h->cfg.n_cond : h->Nq;
   if (n > 0) {
     if (!k_out || !v_out) return WS_ERR_ARG;
     if (!aligned16(k_out) || !aligned16(v_out)) return WS_ERR_ALIGN;
   }
-  const int st = resident(h, unit);
+  const int st = resident(h, session, unit);
   if (st != WS_OK) return st;
   const size_t slot = (size_t)(unit % h->C);
-  if (seg == WS_SEG_LATENT && !h->latent_ready[slot * h->cfg.n_layers + layer]) return WS_ERR_NOT_READY;
+  if (seg == WS_SEG_LATENT && !h->rings[(size_t)session].latent_ready[slot * h->cfg.n_layers + layer])
+    return WS_ERR_NOT_READY;
   ReadParams p{};
   p.cache = h->kv;
   p.dst_k = k_out;
@@ -414,14 +474,33 @@ int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg, uint16_t* k_o
   p.n_tokens = n;
   p.n_heads = h->cfg.n_heads;
   p.head_dim = h->cfg.head_dim;
-  p.plane_rows = (int64_t)h->C * h->T;
-  p.row0 = (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  p.plane_rows = h->session_rows * h->n_sessions;
+  p.row0 = session * h->session_rows + (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
   return cuda_status(launch_read(p, stream));
 }
 
+int ws_cache_read(ws_cache_t* h, int layer, int64_t unit, int seg, uint16_t* k_out, uint16_t* v_out,
+                  cudaStream_t stream) {
+  return ws_session_read(h, 0, layer, unit, seg, k_out, v_out, stream);
+}
+
+int ws_session_slot_table(const ws_cache_t* h, int32_t session, int64_t* slot_unit_host) {
+  if (!h || !slot_unit_host || session < 0 || session >= h->n_sessions) return WS_ERR_ARG;
+  const Ring& r = h->rings[(size_t)session];
+  std::copy(r.slot_unit.begin(), r.slot_unit.end(), slot_unit_host);
+  return WS_OK;
+}
+
 int ws_cache_slot_table(const ws_cache_t* h, int64_t* slot_unit_host) {
-  if (!h || !slot_unit_host) return WS_ERR_ARG;
-  std::copy(h->slot_unit.begin(), h->slot_unit.end(), slot_unit_host);
+  return ws_session_slot_table(h, 0, slot_unit_host);
+}
+
+int ws_session_reset(ws_cache_t* h, int32_t session) {
+  if (!h || session < 0 || session >= h->n_sessions) return WS_ERR_ARG;
+  Ring& r = h->rings[(size_t)session];
+  r.newest = -1;
+  std::fill(r.slot_unit.begin(), r.slot_unit.end(), -1);
+  std::fill(r.latent_ready.begin(), r.latent_ready.end(), 0);
   return WS_OK;
 }
 
@@ -430,7 +509,8 @@ int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info) {
   info->slots = h->C;
   info->tokens_per_unit = h->T;
   info->n_query = h->Nq;
-  info->newest_unit = h->newest;
+  info->newest_unit = h->rings[0].newest;
+  info->n_sessions = h->n_sessions;
   info->cache_bytes = h->kv_bytes;
   info->workspace_bytes = h->ws_bytes;
   return WS_OK;

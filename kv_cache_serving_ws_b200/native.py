@@ -42,7 +42,8 @@ class ws_cache_config(C.Structure):
 
 class ws_cache_info(C.Structure):
     _fields_ = [("slots", C.c_int32), ("tokens_per_unit", C.c_int32), ("n_query", C.c_int32),
-                ("newest_unit", C.c_int64), ("cache_bytes", C.c_uint64), ("workspace_bytes", C.c_uint64)]
+                ("newest_unit", C.c_int64), ("cache_bytes", C.c_uint64), ("workspace_bytes", C.c_uint64),
+                ("n_sessions", C.c_int32)]
 
 
 class ws_profile(C.Structure):
@@ -56,7 +57,7 @@ class ws_unit_io(C.Structure):
     _fields_ = [("n_steps", C.c_int32), ("out_per_call", C.c_int32), ("dt", C.c_float), ("n_latent", C.c_int64),
                 ("cond_k", C.c_void_p), ("cond_v", C.c_void_p), ("q", C.c_void_p), ("k_new", C.c_void_p),
                 ("v_new", C.c_void_p), ("out", C.c_void_p), ("x", C.c_void_p), ("vel", C.c_void_p),
-                ("commit_k", C.c_void_p), ("commit_v", C.c_void_p)]
+                ("commit_k", C.c_void_p), ("commit_v", C.c_void_p), ("session", C.c_int32)]
 
 
 class ws_unit_graph_stats(C.Structure):
@@ -100,6 +101,12 @@ def _declare(lib):
         "ws_unit_graph_launch": (C.c_int, [_P, i64, _P]),
         "ws_unit_graph_get_stats": (C.c_int, [_P, C.POINTER(ws_unit_graph_stats)]),
         "ws_unit_graph_destroy": (C.c_int, [_P]),
+        "ws_pool_create": (C.c_int, [C.POINTER(_P), C.POINTER(ws_cache_config), i32, _P]),
+        "ws_session_append": (C.c_int, [_P, i32, i64, C.c_int, _P, _P, _P]),
+        "ws_session_read": (C.c_int, [_P, i32, C.c_int, i64, C.c_int, _P, _P, _P]),
+        "ws_session_slot_table": (C.c_int, [_P, i32, C.POINTER(i64)]),
+        "ws_session_reset": (C.c_int, [_P, i32]),
+        "ws_session_attention": (C.c_int, [_P, C.c_int, i32, C.POINTER(i32), C.POINTER(i64), _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -274,12 +281,51 @@ def ws_attention_noalloc(q, kv, out, n_query, n_keys, n_heads, head_dim, stream=
                                             _stream(stream)), "ws_attention_noalloc", check)
 
 
+def ws_pool_create(cfg: ws_cache_config, n_sessions: int, stream=None, check=True):
+    h = _P()
+    st = lib().ws_pool_create(C.byref(h), C.byref(cfg), int(n_sessions), _stream(stream))
+    _done(st, "ws_pool_create", check)
+    return st, h
+
+
+def ws_session_append(h, session, unit, seg, k_slice, v_slice, stream=None, check=True):
+    return _done(lib().ws_session_append(h, int(session), int(unit), int(seg), _ptr(k_slice), _ptr(v_slice),
+                                         _stream(stream)), "ws_session_append", check)
+
+
+def ws_session_read(h, session, layer, unit, seg, k_out, v_out, stream=None, check=True):
+    return _done(lib().ws_session_read(h, int(session), int(layer), int(unit), int(seg), _ptr(k_out), _ptr(v_out),
+                                       _stream(stream)), "ws_session_read", check)
+
+
+def ws_session_slot_table(h, session) -> list[int]:
+    info = ws_cache_get_info(h)
+    buf = (C.c_int64 * info["slots"])()
+    _done(lib().ws_session_slot_table(h, int(session), buf), "ws_session_slot_table", True)
+    return list(buf)
+
+
+def ws_session_reset(h, session, check=True):
+    return _done(lib().ws_session_reset(h, int(session)), "ws_session_reset", check)
+
+
+def ws_session_attention(h, layer, sessions, units, q, k_new, v_new, out, stream=None, check=True):
+    n = len(sessions)
+    if len(units) != n:
+        raise ValueError("sessions and units differ in length")
+    s_arr = (C.c_int32 * max(1, n))(*[int(s) for s in sessions])
+    u_arr = (C.c_int64 * max(1, n))(*[int(u) for u in units])
+    st = lib().ws_session_attention(h, int(layer), n, s_arr, u_arr, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out),
+                                    _stream(stream))
+    return _done(st, "ws_session_attention", check)
+
+
 def ws_unit_graph_create(h, n_steps, dt, cond_k, cond_v, q, k_new, v_new, out, x, vel, commit_k, commit_v,
-                         out_per_call=True, n_latent=None, check=True):
+                         out_per_call=True, n_latent=None, session=0, check=True):
     """Unit program over cache h; the tensors must stay alive (and in place) while it exists."""
     io = ws_unit_io(int(n_steps), 1 if out_per_call else 0, float(dt), int(x.numel() if n_latent is None else n_latent),
                     _ptr(cond_k), _ptr(cond_v), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(x), _ptr(vel),
-                    _ptr(commit_k), _ptr(commit_v))
+                    _ptr(commit_k), _ptr(commit_v), int(session))
     g = _P()
     st = lib().ws_unit_graph_create(C.byref(g), h, C.byref(io))
     _done(st, "ws_unit_graph_create", check)

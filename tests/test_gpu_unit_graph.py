@@ -68,7 +68,7 @@ def run_direct(h, u, d):
 class Program:
     """Fixed device buffers of a unit program, refilled per unit."""
 
-    def __init__(self, h):
+    def __init__(self, h, session=0):
         c = CFG
         e = lambda *s: torch.empty(s, dtype=torch.bfloat16, device="cuda")
         self.cond_k = e(c.n_layers, c.n_cond, c.n_heads, c.head_dim)
@@ -80,7 +80,8 @@ class Program:
         self.vel = e(STEPS, N_LAT)
         self.x = e(N_LAT)
         _, self.g = ws.ws_unit_graph_create(h, STEPS, DT, self.cond_k, self.cond_v, self.q, self.k_new, self.v_new,
-                                            self.out, self.x, self.vel, self.commit_k, self.commit_v)
+                                            self.out, self.x, self.vel, self.commit_k, self.commit_v,
+                                            session=session)
 
     def load(self, d):
         for name in ("cond_k", "cond_v", "q", "k_new", "v_new", "commit_k", "commit_v", "vel", "x"):
@@ -194,3 +195,36 @@ def test_unit_program_rejects_bad_buffers():
     assert st == ws.WS_ERR_ARG
     prog.close()
     ws.ws_cache_destroy(h)
+
+
+@pytest.mark.gpu
+def test_unit_program_on_one_session_of_a_pool():
+    """A program on session 1 of a two-session pool gives, bit for bit, what direct calls
+    on a plain cache give; session 0's stream in the same pool is left as it was."""
+    require_gpu()
+    c = CFG
+    h_direct = new_cache()
+    _, pool = ws.ws_pool_create(ws.make_config(c.n_layers, c.n_heads, c.head_dim, c.n_video, c.n_audio, c.n_cond,
+                                               c.history_units), 2)
+    other = UnitData(999, 50)
+    ws.ws_session_append(pool, 0, 50, ws.WS_SEG_COND, to_dev(other.cond_k), to_dev(other.cond_v))
+    ws.ws_session_append(pool, 0, 50, ws.WS_SEG_LATENT, to_dev(other.commit_k), to_dev(other.commit_v))
+    prog = Program(pool, session=1)
+    for u in range(6):
+        d = UnitData(31, u)
+        out_d, x_d = run_direct(h_direct, u, d)
+        prog.load(d)
+        ws.ws_unit_graph_launch(prog.g, u)
+        torch.cuda.synchronize()
+        assert np.array_equal(from_dev(prog.out), from_dev(out_d)), u
+        assert np.array_equal(from_dev(prog.x), from_dev(x_d)), u
+    assert ws.ws_session_slot_table(pool, 1) == ws.ws_cache_slot_table(h_direct)
+    assert ws.ws_session_slot_table(pool, 0) == [-1, -1, 50, -1]
+    for l in range(c.n_layers):
+        k = torch.empty((c.n_query, c.n_heads, c.head_dim), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        ws.ws_session_read(pool, 0, l, 50, ws.WS_SEG_LATENT, k, v)
+        assert np.array_equal(from_dev(k), other.commit_k[l]) and np.array_equal(from_dev(v), other.commit_v[l])
+    prog.close()
+    ws.ws_cache_destroy(pool)
+    ws.ws_cache_destroy(h_direct)
