@@ -257,7 +257,7 @@ def run_ours(args, rank, local_rank, world):
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": traffic,
                 "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
-    launches_per_step = (2 + L * S * (2 + (1 if prof["last_n_split"] > 1 else 0)) + S)
+    launches_per_step = 2 + L * S * 2 + S          # conditioning, commit; latent write + attention; Euler
 
     # ---- HBM-bound kernels, timed on their own on the same stream
     extra = hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit)
@@ -697,7 +697,7 @@ def run_schedule(args):
             "mode": "schedule", "workload": w.name, "units": n, "unit_budget_ms": period_s * 1e3,
             "tflop_per_unit": round(flops_unit / 1e12, 2),
             "direct": {"unit_ms": percentiles(per_direct), "host_ms_per_unit": round(host_direct, 3),
-                       "launches_per_unit": 2 + L * S * 3 + S},
+                       "launches_per_unit": 2 + L * S * 2 + S},
             "graph": {"unit_ms": percentiles(per_graph), "host_ms_per_unit": round(host_graph, 3),
                       "record_ms_per_unit": round((s1["record_ms"] - s0["record_ms"]) / max(1, n + 3), 3),
                       "kernel_nodes": s1["nodes"], "updates_in_place": upd, "instantiations": inst,

@@ -202,8 +202,9 @@ int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info);
  * ws_cache_set_splits -- work decomposition of each attention call.  The
  * attention kernel is persistent: one lane of CTAs per pair of 128-row query
  * tiles; the CTAs of a lane share out its (head, key tile) iterations in equal
- * contiguous ranges, and the heads whose range is cut between two CTAs are
- * merged from fp32 partials by a second kernel.  n_split = CTAs per lane:
+ * contiguous ranges.  A (head, query pair) item whose range is cut between
+ * CTAs is written as fp32 partials, and the last CTA to finish a share of it
+ * merges them in the same launch.  n_split = CTAs per lane:
  * 0 = automatic (one CTA per SM over all lanes), 1..1024 forces that count
  * (reduced if the partials would not fit the workspace).
  */
@@ -222,8 +223,10 @@ const char* ws_status_string(int status);
 /*
  * Launch accounting of the attention path, for benchmarks.  While enabled, the
  * library records a CUDA event pair around each attention kernel and each
- * merge kernel (combine_*) it launches (on the caller's stream).  ws_profile_read
+ * latent write it launches (on the caller's stream).  ws_profile_read
  * synchronises those events and returns the totals since the last reset.
+ * combine_*: merges of cut items run inside the attention kernel, so these stay
+ * 0 (kept for layout compatibility).
  */
 typedef struct {
   int64_t attention_launches;

@@ -12,7 +12,8 @@
 // tile of each run masks the rows past its end.
 //
 // Persistent kernel, one CTA per SM, stream-K style: every CTA gets the same
-// number of (Q block, head, key tile) iterations (see Decomp).  A CTA works on a
+// number of (Q block, head, key tile) iterations (see Decomp); an item cut
+// between CTAs is merged by whichever of them finishes its share last.  A CTA works on a
 // block of two 128-row query tiles of one head at a time:
 //   warpgroup 0, 1  softmax of query tile 0 and 1: one query row per thread (=
 //              one TMEM lane); fp32 online softmax in base 2 with a lazily moved
@@ -163,6 +164,58 @@ __device__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) 
     if ((it & 31u) == 31u && global_timer_ns() - t0 > timeout_ns) return false;
   }
   return false;
+}
+
+// Merge of the partials of one row of an item cut between CTAs:
+//   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
+// Piece k was written by CTA c_first + k of the lane: its last item for k = 0
+// (unless the item starts exactly at that CTA's range), its first item
+// otherwise.  The partials were written by other SMs in this launch: read them
+// through L2 only.
+template <int D>
+__device__ __noinline__ void merge_row(const AttnParams& p, int lane_i, int c_first, int pieces, int end0, int r,
+                                       uint16_t* dst) {
+  float m_all = -INFINITY;
+  for (int k = 0; k < pieces; ++k) {
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    m_all = fmaxf(m_all, __ldcg(p.part_ml + (slot * kItemRows + r) * 2));
+  }
+  float l_all = 0.f;
+  for (int k = 0; k < pieces; ++k) {
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot * kItemRows + r) * 2));
+    l_all += ex2_approx(ml.x - m_all) * ml.y;
+  }
+  const float inv = 1.f / l_all;
+#pragma unroll 1
+  for (int c = 0; c < D; c += 32) {
+    float acc[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+    for (int k = 0; k < pieces; ++k) {
+      const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+      const size_t prow = slot * kItemRows + r;
+      const float w = ex2_approx(__ldcg(p.part_ml + prow * 2) - m_all);
+      const float4* po = reinterpret_cast<const float4*>(p.part_o + prow * D + c);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const float4 o = __ldcg(po + q);
+        acc[4 * q + 0] += w * o.x;
+        acc[4 * q + 1] += w * o.y;
+        acc[4 * q + 2] += w * o.z;
+        acc[4 * q + 3] += w * o.w;
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 32; k += 8) {
+      uint4 v;
+      v.x = pack_bf16x2(acc[k + 0] * inv, acc[k + 1] * inv);
+      v.y = pack_bf16x2(acc[k + 2] * inv, acc[k + 3] * inv);
+      v.z = pack_bf16x2(acc[k + 4] * inv, acc[k + 5] * inv);
+      v.w = pack_bf16x2(acc[k + 6] * inv, acc[k + 7] * inv);
+      *reinterpret_cast<uint4*>(dst + c + k) = v;
+    }
+  }
 }
 
 template <int D>
@@ -471,6 +524,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kOFree + a]);
+        if (pieces > 1) {
+          // Stream-K fix-up: the last piece of the item to arrive merges these 32
+          // rows from the pieces' partials (counted per warp: no block barrier).
+          __threadfence();
+          __syncwarp();
+          const size_t ci =
+              ((((size_t)it.j * d.n_qtiles + it.qt()) * p.n_heads + it.h) * kQTiles + a) * 4 + (warp & 3);
+          int last = 0;
+          if (lane == 0) last = atomicAdd(p.fix_count + ci, 1) == pieces - 1;
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            if (lane == 0) p.fix_count[ci] = 0;
+            __threadfence();
+            if (in_unit) merge_row<D>(p, lane_i, c_first, pieces, end0, a * kBlockM + row, dst);
+          }
+        }
       }
     }
   }
@@ -480,60 +549,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
-  }
-}
-
-// Merge of the partials of an item cut between CTAs:
-//   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
-// One warp per (row, head); each lane owns D/32 consecutive columns.
-template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ AttnParams p) {
-  constexpr int kPer = D / 32;
-  const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
-  const int lane = threadIdx.x & 31;
-  const int rows = p.qu.n_units * p.qu.rows;
-  if (gw >= rows * p.n_heads) return;
-  const int row = gw / p.n_heads;
-  const int h = gw - row * p.n_heads;
-  const int j = row / p.qu.rows;
-  const int r_unit = row - j * p.qu.rows;
-  const int qt = r_unit / kItemRows;
-  const int r = r_unit - qt * kItemRows;
-  int lane_i, c_first, pieces, end0;
-  item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
-  if (pieces == 1) return;                       // written directly by its CTA
-  // piece k was written by CTA c_first + k: its last item for k = 0 (unless
-  // the item starts exactly at that CTA's range), its first item otherwise
-  float m_all = -INFINITY;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    m_all = fmaxf(m_all, p.part_ml[(slot * kItemRows + r) * 2]);
-  }
-  float l_all = 0.f;
-  float acc[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    const size_t prow = slot * kItemRows + r;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
-    const float w = ex2_approx(ml.x - m_all);
-    l_all += w * ml.y;
-    const float* po = p.part_o + prow * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 o = *reinterpret_cast<const float4*>(po);
-      acc[0] += w * o.x; acc[1] += w * o.y; acc[2] += w * o.z; acc[3] += w * o.w;
-    } else {
-      const float2 o = *reinterpret_cast<const float2*>(po);
-      acc[0] += w * o.x; acc[1] += w * o.y;
-    }
-  }
-  const float inv = 1.f / l_all;
-  uint16_t* dst = p.out + ((size_t)row * p.n_heads + h) * D + lane * kPer;
-  if constexpr (kPer == 4) {
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
 }
 
@@ -610,18 +625,6 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
   if (head_dim == 128) return launch_attention_d<128>(q_map, kv_map, p, ctas, stream);
   if (head_dim == 64) return launch_attention_d<64>(q_map, kv_map, p, ctas, stream);
   return cudaErrorInvalidValue;
-}
-
-cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  const long long warps = (long long)p.qu.n_units * p.qu.rows * p.n_heads;
-  const int grid = (int)((warps * 32 + 255) / 256);
-  if (head_dim == 128)
-    merge_kernel<128><<<grid, 256, 0, stream>>>(p);
-  else if (head_dim == 64)
-    merge_kernel<64><<<grid, 256, 0, stream>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
 }
 
 }  // namespace ws

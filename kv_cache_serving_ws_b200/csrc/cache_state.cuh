@@ -64,6 +64,8 @@ struct ws_cache {
   float* part_ml = nullptr;
   size_t ws_bytes = 0;
   int* d_status = nullptr;
+  int* d_fix = nullptr;               // arrival counters of the in-kernel merge of cut items
+  size_t fix_bytes = 0;
   CUtensorMap kv_map;
   int force_lane_ctas = 0;
   int64_t slot_cap = 0;

@@ -89,6 +89,7 @@ struct AttnParams {
   uint16_t* out;            // [n_units * Nq][H][D] bf16
   float* part_o;            // [2 * CTAs][kItemRows][D] fp32
   float* part_ml;           // [2 * CTAs][kItemRows][2] (reference max in log2 units, sum)
+  int* fix_count;           // [fix_counters()] arrivals per (cut item, Q tile, warp); zero between launches
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
   int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)
@@ -110,8 +111,10 @@ void decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced);
 // Partial slots a decomposition needs (two per CTA).
 inline int64_t partial_slots(const Decomp& d) { return (int64_t)d.lanes * d.lane_ctas * 2; }
 
-// Merge of the partials of items shared by several CTAs (no-op for the others).
-cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream);
+// Arrival counters of a call: one per (item, Q tile, warp of its softmax warpgroup).
+inline int64_t fix_counters(int n_units, int n_qtiles, int heads) {
+  return (int64_t)n_units * n_qtiles * heads * kQTiles * 4;
+}
 
 // Copy a [L][n][H][D] token-major slice into the head-major cache planes:
 // plane (l*2 + kv)*H + h, rows row0 .. row0+n-1 of each plane.

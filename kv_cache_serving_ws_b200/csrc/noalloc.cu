@@ -15,13 +15,15 @@
 // Limits and sharing: the array holds kScratchBytes (48 MiB) on every device
 // that loads this part of the library, until the process exits.  The partials
 // take two slots per CTA (at most one CTA per SM unless the query blocks
-// outnumber the SMs): 39 MB at head_dim 128 on 148 SMs.  Requests whose
+// outnumber the SMs): 39 MB at head_dim 128 on 148 SMs; the merge counters
+// (one int per item, Q tile and warp) a few KB more.  Requests whose
 // partials would not fit are rejected with WS_ERR_UNSUPPORTED.  All
 // calls share the array, and it keeps the last call's contents: calls that
 // overlap on the GPU (different streams, or different host threads without
 // ordering) race on it and must be serialised by the caller.  The status word
-// is cleared at the start of every call; the partials need no clearing,
-// because every slot the merge reads is written first by the same call.
+// and the merge counters are cleared at the start of every call; the partials
+// need no clearing, because every slot a merge reads is written first by the
+// same call.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -81,20 +83,22 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   p.runs.rows[0] = n_keys;
   p.runs.tile_begin[0] = 0;
 
-  // scratch layout: [status | part_ml | part_o], two partial slots per CTA
+  // scratch layout: [status | merge counters | part_ml | part_o], two partial slots per CTA
   const int n_qtiles = (n_query + kItemRows - 1) / kItemRows;
   decompose(p.dec, n_qtiles, n_heads, p.qu.tile_start[1], 0);
   const size_t slots = (size_t)partial_slots(p.dec);
   const size_t slot_bytes = (size_t)kItemRows * (head_dim + 2) * sizeof(float);
-  if (kStatusBytes + slots * slot_bytes > kScratchBytes) return WS_ERR_UNSUPPORTED;
+  const size_t fix_bytes = ((size_t)fix_counters(1, n_qtiles, n_heads) * sizeof(int) + 255) & ~(size_t)255;
+  if (kStatusBytes + fix_bytes + slots * slot_bytes > kScratchBytes) return WS_ERR_UNSUPPORTED;
 
   void* base = nullptr;
   const int st = scratch_address(&base);
   if (st != WS_OK) return st;
   unsigned char* b = static_cast<unsigned char*>(base);
   p.status = reinterpret_cast<int*>(b);
-  p.part_ml = reinterpret_cast<float*>(b + kStatusBytes);
-  p.part_o = reinterpret_cast<float*>(b + kStatusBytes + slots * kItemRows * 2 * sizeof(float));
+  p.fix_count = reinterpret_cast<int*>(b + kStatusBytes);
+  p.part_ml = reinterpret_cast<float*>(b + kStatusBytes + fix_bytes);
+  p.part_o = reinterpret_cast<float*>(b + kStatusBytes + fix_bytes + slots * kItemRows * 2 * sizeof(float));
 
   p.n_heads = n_heads;
   p.plane_k = 0;
@@ -108,15 +112,8 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
   if (encode_q_map(&q_map, q, head_dim, n_heads, n_query) != 0) return WS_ERR_CUDA;
   if (encode_kv_map(&kv_map, kv, head_dim, n_keys, (int64_t)2 * n_heads) != 0) return WS_ERR_CUDA;
 
-  if (cudaMemsetAsync(p.status, 0, sizeof(int), stream) != cudaSuccess) return WS_ERR_CUDA;
+  // the status word and the merge counters start at zero (a call that gave up may have left them set)
+  if (cudaMemsetAsync(p.status, 0, kStatusBytes + fix_bytes, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (launch_attention(q_map, kv_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
-  bool any_split = false;
-  for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
-    for (int h = 0; h < n_heads && !any_split; ++h) {
-      int lane, c_first, pieces, end0;
-      item_span(p.dec, p.qu, 0, qt, h, lane, c_first, pieces, end0);
-      any_split = pieces > 1;
-    }
-  if (any_split && launch_merge(p, head_dim, stream) != cudaSuccess) return WS_ERR_CUDA;
   return WS_OK;
 }

@@ -112,6 +112,7 @@ void free_all(ws_cache* h) {
   if (h->part_o) cudaFree(h->part_o);
   if (h->part_ml) cudaFree(h->part_ml);
   if (h->d_status) cudaFree(h->d_status);
+  if (h->d_fix) cudaFree(h->d_fix);
   h->ev_attn.destroy();
   h->ev_comb.destroy();
   h->ev_lat.destroy();
@@ -203,15 +204,6 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   while (partial_slots(p.dec) > h->slot_cap && p.dec.lane_ctas > 1)
     decompose(p.dec, n_qtiles, H, tiles, std::max(1, p.dec.lane_ctas / 2));
   if (partial_slots(p.dec) > h->slot_cap) return WS_ERR_UNSUPPORTED;
-  bool any_split = false;
-  for (int j = 0; j < n && !any_split; ++j)
-    for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
-      for (int hh = 0; hh < H && !any_split; ++hh) {
-        int lane, c_first, pieces, end0;
-        item_span(p.dec, p.qu, j, qt, hh, lane, c_first, pieces, end0);
-        any_split = pieces > 1;
-      }
-
   CUtensorMap q_map;
   if (encode_q_map(&q_map, q, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
 
@@ -246,6 +238,7 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   p.part_o = h->part_o;
   p.part_ml = h->part_ml;
   p.status = h->d_status;
+  p.fix_count = h->d_fix;
   p.timeout_ns = h->timeout_ns;
   p.debug_skip_v_tile = h->debug_skip_v_tile;
   cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_attn.next() : nullptr;
@@ -253,12 +246,6 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   int ctas = 0;
   if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
-  if (any_split) {
-    ev = h->profiling && !h->capturing ? h->ev_comb.next() : nullptr;
-    if (ev) cudaEventRecord(ev[0], stream);
-    if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
-    if (ev) cudaEventRecord(ev[1], stream);
-  }
   h->last_split = p.dec.lane_ctas;
   h->last_ctas = ctas;
   h->last_keys = keys;
@@ -377,13 +364,16 @@ int ws_pool_create(ws_cache_t** out, const ws_cache_config* cfg, int32_t n_sessi
   h->slot_cap = 2 * std::max<int64_t>(sm_count(), n_qtiles);
   const size_t part_o_bytes = (size_t)h->slot_cap * kItemRows * D * 4;
   const size_t part_ml_bytes = (size_t)h->slot_cap * kItemRows * 2 * 4;
-  h->ws_bytes = part_o_bytes + part_ml_bytes;
+  h->fix_bytes = (size_t)fix_counters(kMaxQUnits, (int)n_qtiles, H) * sizeof(int);
+  h->ws_bytes = part_o_bytes + part_ml_bytes + h->fix_bytes;
   int st = WS_OK;
   if (cudaMalloc(&h->kv, h->kv_bytes) != cudaSuccess || cudaMalloc(&h->part_o, part_o_bytes) != cudaSuccess ||
-      cudaMalloc(&h->part_ml, part_ml_bytes) != cudaSuccess || cudaMalloc(&h->d_status, sizeof(int)) != cudaSuccess)
+      cudaMalloc(&h->part_ml, part_ml_bytes) != cudaSuccess || cudaMalloc(&h->d_status, sizeof(int)) != cudaSuccess ||
+      cudaMalloc(&h->d_fix, h->fix_bytes) != cudaSuccess)
     st = WS_ERR_OOM;
   if (st == WS_OK && (cudaMemsetAsync(h->kv, 0, h->kv_bytes, stream) != cudaSuccess ||
-                      cudaMemsetAsync(h->d_status, 0, sizeof(int), stream) != cudaSuccess))
+                      cudaMemsetAsync(h->d_status, 0, sizeof(int), stream) != cudaSuccess ||
+                      cudaMemsetAsync(h->d_fix, 0, h->fix_bytes, stream) != cudaSuccess))
     st = WS_ERR_CUDA;
   if (st == WS_OK && encode_kv_map(&h->kv_map, h->kv, D, rows, (int64_t)L * 2 * H) != 0) st = WS_ERR_CUDA;
   if (st != WS_OK) {
@@ -534,7 +524,9 @@ int ws_sync(ws_cache_t* h, cudaStream_t stream) {
   int s = 0;
   if (cudaMemcpy(&s, h->d_status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return WS_ERR_CUDA;
   if (s != 0) {
+    // a kernel that gave up may have left merge counters mid-count
     if (cudaMemset(h->d_status, 0, sizeof(int)) != cudaSuccess) return WS_ERR_CUDA;
+    if (cudaMemset(h->d_fix, 0, h->fix_bytes) != cudaSuccess) return WS_ERR_CUDA;
     return WS_ERR_DEVICE_TIMEOUT;
   }
   return WS_OK;
