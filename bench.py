@@ -257,7 +257,8 @@ def run_ours(args, rank, local_rank, world):
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": traffic,
                 "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
-    launches_per_step = 2 + L * S * 2 + S          # conditioning, commit; latent write + attention; Euler
+    # conditioning, commit; latent write + attention per call; Euler; separate merges if any
+    launches_per_step = 2 + L * S * 2 + S + prof["combine_launches"] // max(1, args.steps)
 
     # ---- HBM-bound kernels, timed on their own on the same stream
     extra = hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit)

@@ -203,8 +203,9 @@ int ws_cache_get_info(const ws_cache_t* h, ws_cache_info* info);
  * attention kernel is persistent: one lane of CTAs per pair of 128-row query
  * tiles; the CTAs of a lane share out its (head, key tile) iterations in equal
  * contiguous ranges.  A (head, query pair) item whose range is cut between
- * CTAs is written as fp32 partials, and the last CTA to finish a share of it
- * merges them in the same launch.  n_split = CTAs per lane:
+ * CTAs is written as fp32 partials and merged: by the last CTA to finish a
+ * share of it, in the same launch, when every CTA runs at least 64 iterations,
+ * else by a second, short kernel.  n_split = CTAs per lane:
  * 0 = automatic (one CTA per SM over all lanes), 1..1024 forces that count
  * (reduced if the partials would not fit the workspace).
  */
@@ -223,10 +224,10 @@ const char* ws_status_string(int status);
 /*
  * Launch accounting of the attention path, for benchmarks.  While enabled, the
  * library records a CUDA event pair around each attention kernel and each
- * latent write it launches (on the caller's stream).  ws_profile_read
- * synchronises those events and returns the totals since the last reset.
- * combine_*: merges of cut items run inside the attention kernel, so these stay
- * 0 (kept for layout compatibility).
+ * latent write and merge kernel (combine_*) it launches (on the caller's
+ * stream); calls that merge inside the attention kernel launch no merge.
+ * ws_profile_read synchronises those events and returns the totals since the
+ * last reset.
  */
 typedef struct {
   int64_t attention_launches;

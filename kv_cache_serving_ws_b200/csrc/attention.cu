@@ -175,16 +175,29 @@ __device__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) 
 template <int D>
 __device__ __noinline__ void merge_row(const AttnParams& p, int lane_i, int c_first, int pieces, int end0, int r,
                                        uint16_t* dst) {
+  constexpr int kCached = 8;                 // pieces whose (m, l) stay in registers
+  auto row_of = [&](int k) -> size_t {
+    return partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0) * kItemRows + r;
+  };
+  // every piece's (reference max, sum): independent loads, one round trip
+  float2 ml[kCached];
   float m_all = -INFINITY;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    m_all = fmaxf(m_all, __ldcg(p.part_ml + (slot * kItemRows + r) * 2));
+#pragma unroll
+  for (int k = 0; k < kCached; ++k) {
+    ml[k] = k < pieces ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + row_of(k) * 2)) : make_float2(-INFINITY, 0.f);
+    m_all = fmaxf(m_all, ml[k].x);
   }
+  for (int k = kCached; k < pieces; ++k) m_all = fmaxf(m_all, __ldcg(p.part_ml + row_of(k) * 2));
+  float w[kCached];
   float l_all = 0.f;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    const float2 ml = __ldcg(reinterpret_cast<const float2*>(p.part_ml + (slot * kItemRows + r) * 2));
-    l_all += ex2_approx(ml.x - m_all) * ml.y;
+#pragma unroll
+  for (int k = 0; k < kCached; ++k) {
+    w[k] = k < pieces ? ex2_approx(ml[k].x - m_all) : 0.f;
+    l_all += w[k] * ml[k].y;
+  }
+  for (int k = kCached; k < pieces; ++k) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(p.part_ml + row_of(k) * 2));
+    l_all += ex2_approx(v.x - m_all) * v.y;
   }
   const float inv = 1.f / l_all;
 #pragma unroll 1
@@ -192,18 +205,26 @@ __device__ __noinline__ void merge_row(const AttnParams& p, int lane_i, int c_fi
     float acc[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-    for (int k = 0; k < pieces; ++k) {
-      const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-      const size_t prow = slot * kItemRows + r;
-      const float w = ex2_approx(__ldcg(p.part_ml + prow * 2) - m_all);
-      const float4* po = reinterpret_cast<const float4*>(p.part_o + prow * D + c);
+    // two pieces' 32 columns in flight per round trip
+#pragma unroll 1
+    for (int k = 0; k < pieces; k += 2) {
+      const bool two = k + 1 < pieces;
+      const float4* p0 = reinterpret_cast<const float4*>(p.part_o + row_of(k) * D + c);
+      const float4* p1 = reinterpret_cast<const float4*>(p.part_o + row_of(two ? k + 1 : k) * D + c);
+      float4 o0[8], o1[8];
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
-        const float4 o = __ldcg(po + q);
-        acc[4 * q + 0] += w * o.x;
-        acc[4 * q + 1] += w * o.y;
-        acc[4 * q + 2] += w * o.z;
-        acc[4 * q + 3] += w * o.w;
+        o0[q] = __ldcg(p0 + q);
+        o1[q] = two ? __ldcg(p1 + q) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+      const float w0 = k < kCached ? w[k] : ex2_approx(__ldcg(p.part_ml + row_of(k) * 2) - m_all);
+      const float w1 = !two ? 0.f : (k + 1 < kCached ? w[k + 1] : ex2_approx(__ldcg(p.part_ml + row_of(k + 1) * 2) - m_all));
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        acc[4 * q + 0] += w0 * o0[q].x + w1 * o1[q].x;
+        acc[4 * q + 1] += w0 * o0[q].y + w1 * o1[q].y;
+        acc[4 * q + 2] += w0 * o0[q].z + w1 * o1[q].z;
+        acc[4 * q + 3] += w0 * o0[q].w + w1 * o1[q].w;
       }
     }
 #pragma unroll
@@ -524,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars[kOFree + a]);
-        if (pieces > 1) {
+        if (pieces > 1 && p.fixup) {
           // Stream-K fix-up: the last piece of the item to arrive merges these 32
           // rows from the pieces' partials (counted per warp: no block barrier).
           __threadfence();
@@ -549,6 +570,61 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Merge of the partials of items cut between CTAs as a separate launch (calls
+// whose CTAs run few iterations, see AttnParams::fixup):
+//   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
+// One warp per (row, head); each lane owns D/32 consecutive columns.
+template <int D>
+__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ AttnParams p) {
+  constexpr int kPer = D / 32;
+  const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int rows = p.qu.n_units * p.qu.rows;
+  if (gw >= rows * p.n_heads) return;
+  const int row = gw / p.n_heads;
+  const int h = gw - row * p.n_heads;
+  const int j = row / p.qu.rows;
+  const int r_unit = row - j * p.qu.rows;
+  const int qt = r_unit / kItemRows;
+  const int r = r_unit - qt * kItemRows;
+  int lane_i, c_first, pieces, end0;
+  item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
+  if (pieces == 1) return;                       // written directly by its CTA
+  // piece k was written by CTA c_first + k: its last item for k = 0 (unless
+  // the item starts exactly at that CTA's range), its first item otherwise
+  float m_all = -INFINITY;
+  for (int k = 0; k < pieces; ++k) {
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    m_all = fmaxf(m_all, p.part_ml[(slot * kItemRows + r) * 2]);
+  }
+  float l_all = 0.f;
+  float acc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
+  for (int k = 0; k < pieces; ++k) {
+    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
+    const size_t prow = slot * kItemRows + r;
+    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
+    const float w = ex2_approx(ml.x - m_all);
+    l_all += w * ml.y;
+    const float* po = p.part_o + prow * D + lane * kPer;
+    if constexpr (kPer == 4) {
+      const float4 o = *reinterpret_cast<const float4*>(po);
+      acc[0] += w * o.x; acc[1] += w * o.y; acc[2] += w * o.z; acc[3] += w * o.w;
+    } else {
+      const float2 o = *reinterpret_cast<const float2*>(po);
+      acc[0] += w * o.x; acc[1] += w * o.y;
+    }
+  }
+  const float inv = 1.f / l_all;
+  uint16_t* dst = p.out + ((size_t)row * p.n_heads + h) * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv));
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
   }
 }
 
@@ -625,6 +701,18 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
   if (head_dim == 128) return launch_attention_d<128>(q_map, kv_map, p, ctas, stream);
   if (head_dim == 64) return launch_attention_d<64>(q_map, kv_map, p, ctas, stream);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
+  const long long warps = (long long)p.qu.n_units * p.qu.rows * p.n_heads;
+  const int grid = (int)((warps * 32 + 255) / 256);
+  if (head_dim == 128)
+    merge_kernel<128><<<grid, 256, 0, stream>>>(p);
+  else if (head_dim == 64)
+    merge_kernel<64><<<grid, 256, 0, stream>>>(p);
+  else
+    return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 }  // namespace ws

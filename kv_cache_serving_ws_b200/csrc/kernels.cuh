@@ -90,6 +90,7 @@ struct AttnParams {
   float* part_o;            // [2 * CTAs][kItemRows][D] fp32
   float* part_ml;           // [2 * CTAs][kItemRows][2] (reference max in log2 units, sum)
   int* fix_count;           // [fix_counters()] arrivals per (cut item, Q tile, warp); zero between launches
+  int32_t fixup;            // 1: cut items merged inside the kernel; 0: by launch_merge afterwards
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
   int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)
@@ -111,6 +112,13 @@ void decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced);
 // Partial slots a decomposition needs (two per CTA).
 inline int64_t partial_slots(const Decomp& d) { return (int64_t)d.lanes * d.lane_ctas * 2; }
 
+// Merge of cut items as its own launch (when p.fixup == 0).
+cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream);
+// In-kernel merging pays a fence and an atomic per cut item on the CTA's path and
+// puts the last merge on the kernel's tail: worth it once a CTA runs this many
+// iterations (the separate merge launch then costs more).
+constexpr long long kFixupMinIterations = 64;
+inline bool use_fixup(const Decomp& d) { return lane_per(d, 0) >= kFixupMinIterations; }
 // Arrival counters of a call: one per (item, Q tile, warp of its softmax warpgroup).
 inline int64_t fix_counters(int n_units, int n_qtiles, int heads) {
   return (int64_t)n_units * n_qtiles * heads * kQTiles * 4;

@@ -114,6 +114,15 @@ extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint1
 
   // the status word and the merge counters start at zero (a call that gave up may have left them set)
   if (cudaMemsetAsync(p.status, 0, kStatusBytes + fix_bytes, stream) != cudaSuccess) return WS_ERR_CUDA;
+  p.fixup = use_fixup(p.dec) ? 1 : 0;
   if (launch_attention(q_map, kv_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
+  bool any_split = false;
+  for (int qt = 0; qt < n_qtiles && !any_split && !p.fixup; ++qt)
+    for (int h = 0; h < n_heads && !any_split; ++h) {
+      int lane, c_first, pieces, end0;
+      item_span(p.dec, p.qu, 0, qt, h, lane, c_first, pieces, end0);
+      any_split = pieces > 1;
+    }
+  if (any_split && launch_merge(p, head_dim, stream) != cudaSuccess) return WS_ERR_CUDA;
   return WS_OK;
 }

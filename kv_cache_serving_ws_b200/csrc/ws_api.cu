@@ -204,6 +204,16 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   while (partial_slots(p.dec) > h->slot_cap && p.dec.lane_ctas > 1)
     decompose(p.dec, n_qtiles, H, tiles, std::max(1, p.dec.lane_ctas / 2));
   if (partial_slots(p.dec) > h->slot_cap) return WS_ERR_UNSUPPORTED;
+  p.fixup = use_fixup(p.dec) ? 1 : 0;
+  bool any_split = false;
+  for (int j = 0; j < n && !any_split && !p.fixup; ++j)
+    for (int qt = 0; qt < n_qtiles && !any_split; ++qt)
+      for (int hh = 0; hh < H && !any_split; ++hh) {
+        int lane, c_first, pieces, end0;
+        item_span(p.dec, p.qu, j, qt, hh, lane, c_first, pieces, end0);
+        any_split = pieces > 1;
+      }
+
   CUtensorMap q_map;
   if (encode_q_map(&q_map, q, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
 
@@ -246,6 +256,12 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   int ctas = 0;
   if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
+  if (any_split) {
+    ev = h->profiling && !h->capturing ? h->ev_comb.next() : nullptr;
+    if (ev) cudaEventRecord(ev[0], stream);
+    if (launch_merge(p, D, stream) != cudaSuccess) return WS_ERR_CUDA;
+    if (ev) cudaEventRecord(ev[1], stream);
+  }
   h->last_split = p.dec.lane_ctas;
   h->last_ctas = ctas;
   h->last_keys = keys;

@@ -157,3 +157,22 @@ def test_wrapped_ring_many_tiles_and_determinism():
     got2, _ = p.attend(0, 9, splits=0)
     assert np.array_equal(got1, got2)            # same inputs, same launch: same bits
     p.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("splits,heads", [(12, 1), (3, 2)])
+def test_long_history_items_merged_inside_the_kernel(splits, heads):
+    """Long items (a 512-unit window, 1 024 key tiles per head) cut into many pieces,
+    with at least 64 iterations per CTA: the cut items are merged inside the
+    attention kernel (12 pieces also exceed the merge's register-held (max, sum)
+    cache).  One query block, 256 rows."""
+    require_gpu()
+    cfg = orc.Config(n_layers=1, n_heads=heads, head_dim=128, n_video=250, n_audio=6, n_cond=0, history_units=511)
+    p = Pair(cfg, seed=23)
+    for u in range(511):
+        p.cond(u)
+        p.commit(u)
+    p.cond(511)
+    got, want = p.attend(0, 511, splits=splits)
+    _check(got, want)
+    p.close()
