@@ -54,3 +54,49 @@ def test_inject_hook_validates_its_argument():
     assert ws.ws_debug_inject_stall(h, -2, check=False) == ws.WS_ERR_ARG
     assert ws.ws_debug_inject_stall(None, 0, check=False) == ws.WS_ERR_ARG
     ws.ws_cache_destroy(h)
+
+
+@pytest.mark.gpu
+def test_timeout_during_an_in_kernel_merge_leaves_no_stale_counters(monkeypatch):
+    """A call long enough to merge its cut items inside the kernel (6 CTAs x 171
+    key tiles over 8 items of 128 tiles) stalls at CTA-local tile 150: some CTAs
+    have already counted their piece of a cut item, the others never will.  ws_sync
+    reports the timeout and clears the counters with the status word; the next call
+    merges every item correctly (a stale count would make a CTA merge before the
+    other piece was written)."""
+    require_gpu()
+    monkeypatch.setenv("WS_WAIT_TIMEOUT_MS", "200")
+    H, D, Nv, Na, U = 8, 128, 250, 6, 63
+    Nq = Nv + Na
+    cfg = orc.Config(1, H, D, Nv, Na, 0, U)
+    _, h = ws.ws_cache_create(ws.make_config(1, H, D, Nv, Na, 0, U))
+    o = orc.UnitCache(cfg)
+    bits = lambda kind, shape, u=0: synth.normal_tensor(synth.stream_key(37, kind, u), shape)
+    cs, ls, qs = (1, 0, H, D), (1, Nq, H, D), (Nq, H, D)
+    for u in range(U + 1):
+        k, v = bits(synth.KIND_COND_K, cs, u), bits(synth.KIND_COND_V, cs, u)
+        ws.ws_cache_append(h, u, ws.WS_SEG_COND, to_dev(k), to_dev(v))
+        o.append(u, orc.SEG_COND, k, v)
+        if u < U:
+            k, v = bits(synth.KIND_COMMIT_K, ls, u), bits(synth.KIND_COMMIT_V, ls, u)
+            ws.ws_cache_append(h, u, ws.WS_SEG_LATENT, to_dev(k), to_dev(v))
+            o.append(u, orc.SEG_LATENT, k, v)
+    q, kn, vn = (bits(kd, qs, U) for kd in (synth.KIND_Q, synth.KIND_K_NEW, synth.KIND_V_NEW))
+    out = torch.empty(qs, dtype=torch.bfloat16, device="cuda")
+    ws.ws_cache_set_splits(h, 6)
+    assert ws.ws_sync(h, check=False) == ws.WS_OK
+
+    ws.ws_debug_inject_stall(h, 150)
+    assert ws.ws_unit_attention(h, 0, U, to_dev(q), to_dev(kn), to_dev(vn), out, check=False) == ws.WS_OK
+    assert ws.ws_sync(h, check=False) == ws.WS_ERR_DEVICE_TIMEOUT
+    prof_split = ws.ws_profile_read(h)["last_n_split"]
+    assert prof_split == 6
+
+    ws.ws_debug_inject_stall(h, -1)
+    for _ in range(2):                                   # and once more on clean counters
+        assert ws.ws_unit_attention(h, 0, U, to_dev(q), to_dev(kn), to_dev(vn), out, check=False) == ws.WS_OK
+        assert ws.ws_sync(h, check=False) == ws.WS_OK
+        st, want = o.unit_attention(0, U, q, kn, vn)
+        d = np.abs(dev_f64(out) - want)
+        assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (float(d.max()), float(d.mean()))
+    ws.ws_cache_destroy(h)
