@@ -789,6 +789,86 @@ def run_sessions(args):
             sys.exit(1)
 
 
+def run_configs(args):
+    """Attention of one layer at each configuration of the scope table, one call at a
+    time with L2 flushed before each (a 256 MB write), CUDA events around the call
+    only: 5 warm-up calls, then `calls` timed ones; median and min.  Reports TFLOP/s
+    against the measured burst bf16 peak (a kernel timed alone) and, for the small
+    cases, the byte roofline (K/V read once + Q, k_new, v_new and the output)."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200.workloads import RING, TINY, V01, V02, GpuSession
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for w in (TINY, V01, V02, RING):
+        g = GpuSession(w)
+        g.prefill()
+        q, kn, vn = g.step_inputs(0)
+        out = torch.empty_like(q)
+        for _ in range(5):
+            ws.ws_unit_attention(g.h, 0, w.unit, q, kn, vn, out)
+        times = []
+        for _ in range(args.calls):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ws.ws_unit_attention(g.h, 0, w.unit, q, kn, vn, out)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        st = ws.ws_sync(g.h, check=False)
+        med, mn = statistics.median(times), min(times)
+        flops = w.flops_per_call()
+        kv_bytes = 2 * w.n_keys * w.n_heads * w.head_dim * 2
+        io_bytes = 4 * w.n_query * w.n_heads * w.head_dim * 2
+        t_compute = flops / (pk["bf16"] * 1e12) * 1e3
+        t_memory = (kv_bytes + io_bytes) / (pk["hbm"] * 1e9) * 1e3
+        print(json.dumps({"mode": "configs", "workload": w.name, "calls": args.calls, "l2": "flushed before each call",
+                          "ms_median": round(med, 4), "ms_min": round(mn, 4),
+                          "TFLOP/s": round(flops / med / 1e9, 1),
+                          "frac_of_burst_bf16": round(flops / med / 1e9 / pk["bf16"], 4),
+                          "bytes": kv_bytes + io_bytes, "GB/s": round((kv_bytes + io_bytes) / med / 1e6, 1),
+                          "frac_of_measured_hbm": round((kv_bytes + io_bytes) / med / 1e6 / pk["hbm"], 4),
+                          "roofline_ms": round(max(t_compute, t_memory), 4),
+                          "bound": "tensor" if t_compute >= t_memory else "hbm",
+                          "status": ws.status_string(st)}), flush=True)
+        g.close()
+
+
+def run_euler_sweep(args):
+    """Euler update bandwidth over n = 2^20 .. 2^28 elements (6 bytes moved per
+    element), inputs larger than L2 from 2^25 on, L2 flushed before each call below."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    pk = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    for lg in range(20, 29):
+        n = 1 << lg
+        x = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        v = torch.empty(n, dtype=torch.bfloat16, device="cuda")
+        ws.synth_fill(x, 1000 + lg)
+        ws.synth_fill(v, 2000 + lg)
+        for _ in range(3):
+            ws.ws_flow_step(x, v, 0.25)
+        times = []
+        for _ in range(args.calls):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            ws.ws_flow_step(x, v, 0.25)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        med = statistics.median(times)
+        gbs = 6 * n / med / 1e6
+        print(json.dumps({"mode": "euler_sweep", "n": n, "bytes": 6 * n, "ms_median": round(med, 5),
+                          "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / pk["hbm"], 4),
+                          "frac_of_8TBs": round(gbs / 8000, 4)}), flush=True)
+        del x, v
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -805,6 +885,8 @@ def main():
     ap.add_argument("--schedule", action="store_true",
                     help="per-unit schedule: direct calls vs the unit program, back to back and paced at 160 ms")
     ap.add_argument("--units", type=int, default=24)
+    ap.add_argument("--configs", action="store_true", help="attention of one layer at every configuration, L2 flushed")
+    ap.add_argument("--euler-sweep", action="store_true", help="Euler update bandwidth for n = 2^20 .. 2^28")
     ap.add_argument("--sessions", type=int, default=0,
                     help="concurrent sessions: N conversations batched in one launch vs N launches")
     args = ap.parse_args()
@@ -819,6 +901,12 @@ def main():
         return
     if args.sessions:
         run_sessions(args)
+        return
+    if args.configs:
+        run_configs(args)
+        return
+    if args.euler_sweep:
+        run_euler_sweep(args)
         return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
