@@ -1,5 +1,6 @@
 // Unit program: the device work of one streaming unit (conditioning append,
-// S x L attention calls with their latent writes and merges, S Euler updates,
+// S x L attention calls with their latent writes (and merge launches when a call
+// is too short to merge its cut items in-kernel), S Euler updates,
 // latent commit) recorded as a CUDA graph and replayed once per unit.
 //
 // Each launch records the unit's calls on a private capture stream through the

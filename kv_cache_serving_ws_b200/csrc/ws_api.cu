@@ -125,8 +125,9 @@ namespace ws {
 // Attention of n query units at `layer`: the current unit of several sessions,
 // and/or consecutive units of one session (a prefill).  Writes each unit's
 // k_new/v_new into its latent rows, plans each unit's visible runs in its
-// session's rows, launches the kernel and, when a head's key range was cut
-// between CTAs, the merge.
+// session's rows, and launches the kernel.  Items whose key range is cut
+// between CTAs are merged inside the kernel when every CTA runs a long range,
+// else by a merge launch after it.
 int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_t* units, int n, const uint16_t* q,
                    const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
   if (!h || layer < 0 || layer >= h->cfg.n_layers || !sessions || !units || n < 1) return WS_ERR_ARG;
