@@ -18,8 +18,9 @@
  *   - the flow-matching Euler update of the latent, x <- x + dt*v
  *     (paper.rainbus.top, section 核心方法, flow-matching latent generation).
  *
- * Everything runs on one GPU with no sharding; the pages split the performer
- * across GPUs with Ulysses context parallelism, which this library does not do.
+ * Every call runs on one GPU.  The pages split the performer across GPUs with
+ * Ulysses context parallelism; here that split is a layer above this ABI
+ * (per-rank caches holding a head shard each, exchanges over torch.distributed).
  *
  * Conventions shared by every call
  * --------------------------------
