@@ -1,13 +1,14 @@
 """ws_attention_noalloc -- attention for callers that cannot allocate device memory
 (graph captures without allocation nodes, frameworks that own every allocation,
 real-time loops) -- gives the same result as ws_unit_attention on the same keys,
-for two calls in a row that reuse its shared scratch array with different shapes.
+for calls in a row that reuse its shared scratch array with different shapes, the
+last one long enough to merge its cut items inside the kernel.
 Kept in a file of its own, collected last."""
 import numpy as np
 import pytest
 import torch
 
-from gpu_util import ATOL_MAX, ATOL_MEAN, require_gpu, to_dev
+from gpu_util import ATOL_MAX, ATOL_MEAN, require_gpu
 from kv_cache_serving_ws_b200 import native as ws
 from kv_cache_serving_ws_b200 import synth
 
@@ -17,7 +18,10 @@ def _reference_and_keys(cfg, layer, seed):
     L, H, D, Nv, Na, Nc, U = cfg
     Nq = Nv + Na
     _, h = ws.ws_cache_create(ws.make_config(L, H, D, Nv, Na, Nc, U))
-    bits = lambda kind, shape, u=0, l=0: to_dev(synth.normal_tensor(synth.stream_key(seed, kind, u, l), shape))
+    def bits(kind, shape, u=0, l=0):                 # the device twin of the seeded generator
+        t = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+        ws.synth_fill(t, synth.stream_key(seed, kind, u, l))
+        return t
     unit = U + 1
     for u in range(unit + 1):
         ws.ws_cache_append(h, u, ws.WS_SEG_COND, bits(synth.KIND_COND_K, (L, Nc, H, D), u),
@@ -51,7 +55,10 @@ def _reference_and_keys(cfg, layer, seed):
 def test_noalloc_matches_unit_attention_on_two_calls_in_a_row():
     require_gpu()
     cases = [((2, 6, 128, 250, 4, 16, 3), 1, 21),   # D = 128, key ranges cut between CTAs
-             ((1, 5, 64, 300, 7, 9, 2), 0, 22)]     # D = 64, other shapes: reuses the same scratch
+             ((1, 5, 64, 300, 7, 9, 2), 0, 22),     # D = 64, other shapes: reuses the same scratch
+             # 40 heads x 256 key tiles over 148 CTAs (69 iterations each): cut items are
+             # merged inside the kernel, with the arrival counters in the static array
+             ((1, 40, 128, 250, 6, 0, 127), 0, 23)]
     for cfg, layer, seed in cases:
         q, ref, kv = _reference_and_keys(cfg, layer, seed)
         _, H, D, Nv, Na, _, _ = cfg
