@@ -8,8 +8,18 @@
 #include <cstdint>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/ws.h"
 #include "kernels.cuh"
+
+// An NVTX range around an entry point, for profilers (no cost without one).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 struct EventPool {
   std::vector<cudaEvent_t> ev;   // pairs: 2*i start, 2*i+1 end

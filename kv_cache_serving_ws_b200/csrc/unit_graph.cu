@@ -104,6 +104,7 @@ int ws_unit_graph_create(ws_unit_graph_t** out, ws_cache_t* h, const ws_unit_io*
 }
 
 int ws_unit_graph_launch(ws_unit_graph_t* g, int64_t unit, cudaStream_t stream) {
+  const NvtxRange range("ws_unit_graph_launch");
   if (!g || unit < 0) return WS_ERR_ARG;
   ws_cache* h = g->h;
   const auto t0 = std::chrono::steady_clock::now();

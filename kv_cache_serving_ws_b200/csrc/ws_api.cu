@@ -421,22 +421,26 @@ int ws_cache_destroy(ws_cache_t* h) {
 
 int ws_cache_append(ws_cache_t* h, int64_t unit, int seg, const uint16_t* k_slice, const uint16_t* v_slice,
                     cudaStream_t stream) {
+  const NvtxRange range("ws_cache_append");
   return append_impl(h, 0, unit, seg, k_slice, v_slice, stream);
 }
 
 int ws_session_append(ws_cache_t* h, int32_t session, int64_t unit, int seg, const uint16_t* k_slice,
                       const uint16_t* v_slice, cudaStream_t stream) {
+  const NvtxRange range("ws_session_append");
   return append_impl(h, session, unit, seg, k_slice, v_slice, stream);
 }
 
 int ws_unit_attention(ws_cache_t* h, int layer, int64_t unit, const uint16_t* q, const uint16_t* k_new,
                       const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  const NvtxRange range("ws_unit_attention");
   const int32_t s0 = 0;
   return attention_impl(h, layer, &s0, &unit, 1, q, k_new, v_new, out, stream);
 }
 
 int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n_units, const uint16_t* q,
                          const uint16_t* k_new, const uint16_t* v_new, uint16_t* out, cudaStream_t stream) {
+  const NvtxRange range("ws_prefill_attention");
   if (!h || unit_first < 0 || n_units < 1) return WS_ERR_ARG;
   if (n_units > kMaxQUnits) return WS_ERR_UNSUPPORTED;
   int32_t sess[kMaxQUnits];
@@ -451,15 +455,18 @@ int ws_prefill_attention(ws_cache_t* h, int layer, int64_t unit_first, int32_t n
 int ws_session_attention(ws_cache_t* h, int layer, int32_t n, const int32_t* sessions, const int64_t* units,
                          const uint16_t* q, const uint16_t* k_new, const uint16_t* v_new, uint16_t* out,
                          cudaStream_t stream) {
+  const NvtxRange range("ws_session_attention");
   return attention_impl(h, layer, sessions, units, n, q, k_new, v_new, out, stream);
 }
 
 int ws_flow_step(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream) {
+  const NvtxRange range("ws_flow_step");
   return flow_step_impl(x, v, dt, n, stream);
 }
 
 int ws_session_read(ws_cache_t* h, int32_t session, int layer, int64_t unit, int seg, uint16_t* k_out,
                     uint16_t* v_out, cudaStream_t stream) {
+  const NvtxRange range("ws_session_read");
   if (!h || layer < 0 || layer >= h->cfg.n_layers || unit < 0) return WS_ERR_ARG;
   if (session < 0 || session >= h->n_sessions) return WS_ERR_ARG;
   if (seg != WS_SEG_COND && seg != WS_SEG_LATENT) return WS_ERR_ARG;
@@ -536,6 +543,7 @@ int ws_debug_inject_stall(ws_cache_t* h, int tile) {
 }
 
 int ws_sync(ws_cache_t* h, cudaStream_t stream) {
+  const NvtxRange range("ws_sync");
   if (!h) return WS_ERR_ARG;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return WS_ERR_CUDA;
   int s = 0;
