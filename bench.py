@@ -834,6 +834,67 @@ def run_configs(args):
                           "bound": "tensor" if t_compute >= t_memory else "hbm",
                           "status": ws.status_string(st)}), flush=True)
         g.close()
+        if args.library:
+            for name, res in library_attention(w, args.calls, flush):
+                line = {"mode": "configs", "impl": "library:" + name, "workload": w.name, "calls": args.calls,
+                        "l2": "flushed before each call"}
+                if isinstance(res, str):
+                    line["unavailable"] = res
+                else:
+                    line.update({"ms_median": round(res, 4), "TFLOP/s": round(flops / res / 1e9, 1),
+                                 "frac_of_burst_bf16": round(flops / res / 1e9 / pk["bf16"], 4)})
+                print(json.dumps(line), flush=True)
+
+
+def library_attention(w, calls, flush):
+    """Context for the configurations above: vendor attention kernels timed on dense
+    bf16 N(0,1) tensors of the same sizes (a one-unit query sees every key of its
+    window, so the FLOPs are the same), with the same protocol (L2 flushed, CUDA events
+    around the call, 5 warm-up calls, median).  Never on the product path.  Yields
+    (name, median ms) or (name, reason it could not run)."""
+    import torch
+    import torch.nn.functional as F
+
+    nq, nk, H, D = w.n_query, w.n_keys, w.n_heads, w.head_dim
+
+    def timed(fn):
+        for _ in range(5):
+            fn()
+        ts = []
+        for _ in range(calls):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    gen = torch.Generator(device="cuda").manual_seed(w.seed)
+    q = torch.randn(nq, H, D, device="cuda", dtype=torch.bfloat16, generator=gen)
+    k = torch.randn(nk, H, D, device="cuda", dtype=torch.bfloat16, generator=gen)
+    v = torch.randn(nk, H, D, device="cuda", dtype=torch.bfloat16, generator=gen)
+    try:
+        from torch.nn.attention import SDPBackend, sdpa_kernel
+        qh, kh, vh = (t.transpose(0, 1).unsqueeze(0).contiguous() for t in (q, k, v))
+        with sdpa_kernel([SDPBackend.CUDNN_ATTENTION]):
+            yield "torch-sdpa-cudnn", timed(lambda: F.scaled_dot_product_attention(qh, kh, vh))
+        del qh, kh, vh
+    except Exception as ex:                                   # noqa: BLE001 - reported, not hidden
+        yield "torch-sdpa-cudnn", f"{type(ex).__name__}: {str(ex)[:160]}"
+    for backend in ("cutlass", "cute-dsl"):
+        try:
+            import flashinfer
+            ws_buf = torch.empty(512 << 20, dtype=torch.uint8, device="cuda")
+            fw = flashinfer.BatchPrefillWithRaggedKVCacheWrapper(ws_buf, "NHD", backend=backend)
+            ind = lambda n: torch.tensor([0, n], dtype=torch.int32, device="cuda")
+            fw.plan(ind(nq), ind(nk), H, H, D, causal=False, q_data_type=torch.bfloat16,
+                    kv_data_type=torch.bfloat16)
+            yield "flashinfer-" + backend, timed(lambda: fw.run(q, k, v))
+            del fw, ws_buf
+        except Exception as ex:                               # noqa: BLE001 - reported, not hidden
+            yield "flashinfer-" + backend, f"{type(ex).__name__}: {str(ex)[:160]}"
 
 
 def run_euler_sweep(args):
@@ -886,6 +947,8 @@ def main():
                     help="per-unit schedule: direct calls vs the unit program, back to back and paced at 160 ms")
     ap.add_argument("--units", type=int, default=24)
     ap.add_argument("--configs", action="store_true", help="attention of one layer at every configuration, L2 flushed")
+    ap.add_argument("--library", action="store_true",
+                    help="with --configs: also time vendor attention kernels on dense tensors of the same sizes")
     ap.add_argument("--euler-sweep", action="store_true", help="Euler update bandwidth for n = 2^20 .. 2^28")
     ap.add_argument("--sessions", type=int, default=0,
                     help="concurrent sessions: N conversations batched in one launch vs N launches")

@@ -17,14 +17,18 @@
 // block of two 128-row query tiles of one head at a time:
 //   warpgroup 0, 1  softmax of query tile 0 and 1: one query row per thread (=
 //              one TMEM lane); fp32 online softmax in base 2 with a lazily moved
-//              reference max; P is rounded to bf16 and written back into the TMEM
+//              reference max, taken only when a row's P sum shows it may have to
+//              move; P is rounded to bf16 and written back into the TMEM
 //              columns of its own S (A operand of the P.V product); epilogue of
 //              each item;
 //   warp 8     TMA producer: the two Q tiles of each item, K and V tiles (2 stages);
 //   warp 9     MMA issuer: S_a = Q_a K^T (A and B from shared memory) and
 //              O_a += P_a V (A from TMEM, V as an MN-major B operand), ordered
 //              PV0(j), S0(j+1), PV1(j), S1(j+1): while one warpgroup runs its
-//              softmax the tensor core works on the other tile's products.
+//              softmax the tensor core works on the other tile's products.  The
+//              whole warp runs the issue loop, so descriptors stay warp-uniform,
+//              and one elected lane executes each tcgen05 instruction: issued from
+//              a lone thread, a 128x128x16 MMA took about 85 cycles instead of 64.
 // TMEM: S0 [0,128), O0 [128,128+D), S1 [256,384), O1 [384,384+D).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -155,6 +159,7 @@ struct TileIter {
     flags();
   }
 };
+
 
 // Bounded wait used only to drain in-flight copies and MMAs on the way out.
 __device__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
@@ -348,7 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_v[s] >= 0) drain_wait(&bars[kVFull + s], ((uint32_t)last_v[s] >> 1) & 1, p.timeout_ns);
         }
       }
-    } else if (warp == kMmaWarp && lane == 0) {
+    } else if (warp == kMmaWarp) {
       // -------------------------------------------------------- MMA issuer
       constexpr uint32_t idesc_s = umma_idesc_bf16_f32(kBlockM, kBlockN, false, false);
       constexpr uint32_t idesc_o = umma_idesc_bf16_f32(kBlockM, D, false, true);
@@ -357,8 +362,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_s = [&](const TileIter& it, int a) -> bool {
         const int s = it.g & 1;
         if (a == 0) {
-          if (it.first && !wait_phase(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
-          if (!wait_phase(&bars[kKFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+          if (it.first && !warp_wait(&bars[kQFull], (uint32_t)it.n & 1, guard)) return false;
+          if (!warp_wait(&bars[kKFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
         }
         tc_fence_after_sync();
         const uint32_t d_tmem = tmem_s(tmem, a);
@@ -368,21 +373,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t koff = (uint32_t)((kk >> 2) * kBlockN * kRowBytes + (kk & 3) * 32);
           const uint64_t da = umma_smem_desc_sw128(q_base + a * S::kQTileBytes + off, 16, 1024);
           const uint64_t db = umma_smem_desc_sw128(k_base + s * S::kTileBytes + koff, 16, 1024);
-          umma_bf16_ss(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
+          if (elect_one()) umma_bf16_ss(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bars[kSFull + a]);
+        if (elect_one()) umma_commit(&bars[kSFull + a]);
         if (a == kQTiles - 1) {
-          umma_commit(&bars[kKEmpty + s]);
-          if (it.last) umma_commit(&bars[kQEmpty]);
+          if (elect_one()) umma_commit(&bars[kKEmpty + s]);
+          if (it.last && elect_one()) umma_commit(&bars[kQEmpty]);
         }
         return true;
       };
       // O_a += P_a(g) V(g), P_a in the TMEM columns of S_a, two bf16 per column
       auto issue_pv = [&](const TileIter& it, int a) -> bool {
         const int s = it.g & 1;
-        if (a == 0 && !wait_phase(&bars[kVFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
-        if (!wait_phase(&bars[kPFull + a], (uint32_t)it.g & 1, guard)) return false;
-        if (it.first && it.n > 0 && !wait_phase(&bars[kOFree + a], (uint32_t)(it.n - 1) & 1, guard)) return false;
+        if (a == 0 && !warp_wait(&bars[kVFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+        if (!warp_wait(&bars[kPFull + a], (uint32_t)it.g & 1, guard)) return false;
+        if (it.first && it.n > 0 && !warp_wait(&bars[kOFree + a], (uint32_t)(it.n - 1) & 1, guard)) return false;
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_o(tmem, a);
         const uint32_t p_tmem = tmem_s(tmem, a);
@@ -392,10 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           // head-dim columns one chunk (kBlockN rows) further
           const uint64_t db = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
                                                    kBlockN * kRowBytes, 1024);
-          umma_bf16_ts(o_tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
+          if (elect_one()) umma_bf16_ts(o_tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
         }
-        if (it.last) umma_commit(&bars[kOFull + a]);
-        if (a == kQTiles - 1) umma_commit(&bars[kVEmpty + s]);
+        if (it.last && elect_one()) umma_commit(&bars[kOFull + a]);
+        if (a == kQTiles - 1 && elect_one()) umma_commit(&bars[kVEmpty + s]);
         return true;
       };
       TileIter it_s, it_pv;                  // it_s runs one iteration ahead of it_pv
@@ -411,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && more) ok = issue_s(it_s, 1);
         it_pv.next(p.qu, p.runs);
       }
-      umma_commit(&bars[kMmaDone]);
+      if (elect_one()) umma_commit(&bars[kMmaDone]);
       drain_wait(&bars[kMmaDone], 0, p.timeout_ns);
     }
   } else {
@@ -435,49 +440,100 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait_phase(&bars[kSFull + a], (uint32_t)g & 1, guard);
       if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
       tc_fence_after_sync();
-      uint32_t sr[kBlockN];
-      tmem_load_128(t_s, sr);
       const int valid = it.valid();
-      if (valid < kBlockN) {
-#pragma unroll
-        for (int c = 0; c < kBlockN; ++c)
-          if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row max: 8 independent chains of three-input max
-      float mx[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
-#pragma unroll
-      for (int c = 8; c < kBlockN; c += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
-      const float m_cand =
-          max3_f32(max3_f32(mx[0], mx[1], mx[2]), max3_f32(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) * p.scale_log2;
-      // Move the reference max only when P would exceed 2^8 (or for a new item).
-      const bool move = it.first || m_cand > m_ref + 8.f;
-      float alpha = 1.f;
-      if (move) {
-        alpha = ex2_approx(m_ref - m_cand);
-        l_sum *= alpha;
-        m_ref = m_cand;
-      }
-      // P = 2^(s * log2(e)/sqrt(D) - m): scale and shift on fp32 pairs, one ex2
-      // per element, sums on fp32 pairs (4 independent chains)
       const uint64_t scale2 = f32x2(p.scale_log2, p.scale_log2);
-      const uint64_t negm2 = f32x2(-m_ref, -m_ref);
       uint64_t rs2[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
       uint32_t pk[kBlockN / 2];
+      float alpha = 1.f;
+      bool move = false;
+      // Past an item's first tile the reference max rarely moves, so P is first
+      // computed against the current reference without taking the row max.  The
+      // reference must move only if some P exceeds 2^8, and then the fp32 sum of
+      // the row's P reaches 2^8 too (a rounded sum of positive terms is never
+      // below its largest term; the threshold 255 leaves room for the error of
+      // ex2.approx).  Only a warp with such a row takes the max and recomputes
+      // the tile from S, still intact in TMEM (P is written back after the
+      // check); a row whose own sum triggered it moves its reference to the row
+      // max, so that a slowly rising max cannot trigger a recomputation on every
+      // tile.  Whenever no row sum reaches 255, P, the sums and the reference are
+      // exactly those of taking the max first.
+      bool redo = it.first;
+      bool hot = false;
+      if (!it.first) {
+        uint32_t sr[kBlockN];
+        tmem_load_128(t_s, sr);
+        if (valid < kBlockN) {
 #pragma unroll
-      for (int c = 0; c < kBlockN / 2; ++c) {
-        const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
-        float x0, x1;
-        f32x2_split(x, x0, x1);
-        const float e0 = ex2_approx(x0);
-        const float e1 = ex2_approx(x1);
-        rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
-        pk[c] = pack_bf16x2(e0, e1);
+          for (int c = 0; c < kBlockN; ++c)
+            if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+        }
+        const uint64_t negm2 = f32x2(-m_ref, -m_ref);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kBlockN / 2; ++c) {
+          const float s0 = __uint_as_float(sr[2 * c]), s1 = __uint_as_float(sr[2 * c + 1]);
+          const uint64_t x = fma_f32x2(f32x2(s0, s1), scale2, negm2);
+          float x0, x1;
+          f32x2_split(x, x0, x1);
+          const float e0 = ex2_approx(x0);
+          const float e1 = ex2_approx(x1);
+          rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
+        }
+        float rs[8];
+        f32x2_split(rs2[0], rs[0], rs[1]);
+        f32x2_split(rs2[1], rs[2], rs[3]);
+        f32x2_split(rs2[2], rs[4], rs[5]);
+        f32x2_split(rs2[3], rs[6], rs[7]);
+        const float tile_sum = ((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7]));
+        hot = !(tile_sum < 255.f);
+        redo = __any_sync(0xffffffffu, hot);
+      }
+      if (redo) {
+        uint32_t sr[kBlockN];
+        tmem_load_128(t_s, sr);
+        if (valid < kBlockN) {
+#pragma unroll
+          for (int c = 0; c < kBlockN; ++c)
+            if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
+        }
+        // row max: 8 independent chains of three-input max
+        float mx[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+#pragma unroll
+        for (int c = 8; c < kBlockN; c += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+        const float m_cand =
+            max3_f32(max3_f32(mx[0], mx[1], mx[2]), max3_f32(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
+            p.scale_log2;
+        // Move the reference max when P would exceed 2^8, for a new item, or to
+        // the row max when this row's sum triggered the recomputation.
+        move = it.first || m_cand > m_ref + 8.f || (hot && m_cand > m_ref);
+        if (move) {
+          alpha = ex2_approx(m_ref - m_cand);
+          l_sum *= alpha;
+          m_ref = m_cand;
+        }
+        // P = 2^(s * log2(e)/sqrt(D) - m): scale and shift on fp32 pairs, one ex2
+        // per element, sums on fp32 pairs (4 independent chains)
+        const uint64_t negm2 = f32x2(-m_ref, -m_ref);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
+#pragma unroll
+        for (int c = 0; c < kBlockN / 2; ++c) {
+          const uint64_t x =
+              fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
+          float x0, x1;
+          f32x2_split(x, x0, x1);
+          const float e0 = ex2_approx(x0);
+          const float e1 = ex2_approx(x1);
+          rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
+          pk[c] = pack_bf16x2(e0, e1);
+        }
       }
       float rs[8];
       f32x2_split(rs2[0], rs[0], rs[1]);

@@ -77,6 +77,20 @@ __device__ __forceinline__ bool wait_phase(uint64_t* bar, uint32_t parity, const
   return wait_slow(bar, parity, g);
 }
 
+// A bounded wait taken by every lane of a warp; the result is the same in all
+// lanes, so the warp's control flow stays uniform.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, const WaitGuard& g) {
+  return __all_sync(0xffffffffu, wait_phase(bar, parity, g));
+}
+
+// True in one lane of a converged warp (elect.sync over all 32 lanes): tcgen05
+// instructions issued this way take their operands from warp-uniform values.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}" : "=r"(pred));
+  return pred != 0;
+}
+
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
