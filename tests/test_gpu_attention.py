@@ -176,3 +176,33 @@ def test_long_history_items_merged_inside_the_kernel(splits, heads):
     got, want = p.attend(0, 511, splits=splits)
     _check(got, want)
     p.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("head_dim,splits,slope", [(128, 0, 0.25), (128, 3, 0.25), (64, 0, 0.25), (128, 0, 4.0)])
+def test_rising_scores_move_the_reference_max(head_dim, splits, slope):
+    """Keys scaled by 1 + slope*u for unit u: a row's scores rise tile after tile.
+    With slope 1/4 (scale 1 to 4) the P of a later tile against the earlier reference
+    max often sums past 255 (the row then moves its reference to the row max) or
+    exceeds 2^8 (the lazy move).  With slope 4 (scale up to 49) the scores climb by
+    far more than 128 in log2 units, so a P left against an old reference would
+    overflow to inf: only the check on the P sum, and the move it triggers, keep the
+    output finite.  The tolerance is that of the other stressed-score tests."""
+    require_gpu()
+    cfg = orc.Config(n_layers=1, n_heads=4, head_dim=head_dim, n_video=250, n_audio=6, n_cond=8, history_units=12)
+    p = Pair(cfg, seed=31)
+    scaled = lambda bits, f: orc.f64_to_bf16(orc.bf16_to_f64(bits) * f)
+    for u in range(13):
+        f = 1.0 + slope * u
+        cs = (1, cfg.n_cond, cfg.n_heads, head_dim)
+        k, v = scaled(p._bits(synth.KIND_COND_K, cs, u), f), p._bits(synth.KIND_COND_V, cs, u)
+        assert ws.ws_cache_append(p.h, u, ws.WS_SEG_COND, to_dev(k), to_dev(v), check=False) == 0
+        assert p.o.append(u, orc.SEG_COND, k, v) == 0
+        if u < 12:
+            ls = (1, cfg.n_query, cfg.n_heads, head_dim)
+            k, v = scaled(p._bits(synth.KIND_COMMIT_K, ls, u), f), p._bits(synth.KIND_COMMIT_V, ls, u)
+            assert ws.ws_cache_append(p.h, u, ws.WS_SEG_LATENT, to_dev(k), to_dev(v), check=False) == 0
+            assert p.o.append(u, orc.SEG_LATENT, k, v) == 0
+    got, want = p.attend(0, 12, splits=splits)
+    _check(got, want, max_tol=2e-2, mean_tol=2e-3)
+    p.close()
