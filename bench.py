@@ -930,6 +930,68 @@ def run_euler_sweep(args):
         del x, v
 
 
+def run_hbm_kernels(args):
+    """The HBM-bound kernels at sizes larger than L2 on a small cache (a few GB on the
+    device, so ncu can capture them): the 40-layer latent commit of one 640x368 unit
+    (append_kernel, 1.51 GB moved) into a 40-layer cache with a one-unit history, and
+    the Euler update of 2^28 elements (euler_kernel, 1.61 GB moved).  3 warm-up calls,
+    then `calls` timed ones, each after a 256 MB write that flushes L2; CUDA events
+    around the call only; median."""
+    import torch
+
+    from kv_cache_serving_ws_b200 import native as ws
+    from kv_cache_serving_ws_b200 import synth
+    pk = peaks()
+    L, H, D, Nv, Na, Nc = 40, 40, 128, 920, 4, 32
+    _, h = ws.ws_cache_create(ws.make_config(L, H, D, Nv, Na, Nc, 1))
+    dev = torch.device("cuda")
+    ck = torch.empty((L, Nc, H, D), dtype=torch.bfloat16, device=dev)
+    cv = torch.empty_like(ck)
+    ws.synth_fill(ck, synth.stream_key(8, synth.KIND_COND_K, 0))
+    ws.synth_fill(cv, synth.stream_key(8, synth.KIND_COND_V, 0))
+    ws.ws_cache_append(h, 0, ws.WS_SEG_COND, ck, cv)
+    lk = torch.empty((L, Nv + Na, H, D), dtype=torch.bfloat16, device=dev)
+    lv = torch.empty_like(lk)
+    ws.synth_fill(lk, synth.stream_key(8, synth.KIND_COMMIT_K, 0))
+    ws.synth_fill(lv, synth.stream_key(8, synth.KIND_COMMIT_V, 0))
+    n = 1 << 28
+    x = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    v = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    ws.synth_fill(x, 12345)
+    ws.synth_fill(v, 54321)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(args.calls):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    cases = (("append_kernel", "latent commit, 40 layers x 924 rows x 40 heads x 128, K and V",
+              2 * 2 * lk.numel() * 2, lambda: ws.ws_cache_append(h, 0, ws.WS_SEG_LATENT, lk, lv)),
+             ("euler_kernel", "x <- RN_bf16(x + 0.25 v), 2^28 elements", 6 * n,
+              lambda: ws.ws_flow_step(x, v, 0.25)))
+    for kernel, what, nbytes, fn in cases:
+        ms = timed(fn)
+        gbs = nbytes / ms / 1e6
+        print(json.dumps({"mode": "hbm_kernels", "kernel": kernel, "what": what, "bytes": nbytes,
+                          "calls": args.calls, "l2": "flushed before each call", "ms_median": round(ms, 4),
+                          "GB/s": round(gbs, 1), "frac_of_measured_hbm": round(gbs / pk["hbm"], 4),
+                          "frac_of_8TBs": round(gbs / 8000, 4)}), flush=True)
+    st = ws.ws_sync(h, check=False)
+    ws.ws_cache_destroy(h)
+    if st != ws.WS_OK:
+        sys.exit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -950,6 +1012,8 @@ def main():
     ap.add_argument("--library", action="store_true",
                     help="with --configs: also time vendor attention kernels on dense tensors of the same sizes")
     ap.add_argument("--euler-sweep", action="store_true", help="Euler update bandwidth for n = 2^20 .. 2^28")
+    ap.add_argument("--hbm-kernels", action="store_true",
+                    help="latent commit and Euler update on a small cache, L2 flushed (ncu capture target)")
     ap.add_argument("--sessions", type=int, default=0,
                     help="concurrent sessions: N conversations batched in one launch vs N launches")
     args = ap.parse_args()
@@ -970,6 +1034,9 @@ def main():
         return
     if args.euler_sweep:
         run_euler_sweep(args)
+        return
+    if args.hbm_kernels:
+        run_hbm_kernels(args)
         return
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
