@@ -252,7 +252,9 @@ int ws_profile_read(ws_cache_t* h, ws_profile* out);
  * kernel leaves its loops, drains its copies, frees TMEM and stores
  * WS_ERR_DEVICE_TIMEOUT for ws_sync (the output of that call is undefined).
  * tile = -1 turns it off.  The wait bound is 2 s, or WS_WAIT_TIMEOUT_MS (read
- * when the cache is created).
+ * when the cache is created).  With h = NULL the hook applies to the calls of
+ * ws_attention_noalloc instead (process-wide; their bound is read at each call),
+ * whose status ws_attention_noalloc_sync reports.
  */
 int ws_debug_inject_stall(ws_cache_t* h, int tile);
 
@@ -272,14 +274,14 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit,
 /*
  * ws_attention_noalloc -- block-causal attention for callers that cannot
  * allocate device memory.  The paper has no counterpart: this is an interface
- * for callers that must not call cudaMalloc (inside a CUDA-graph capture that
- * may hold no allocation, under a framework that owns every allocation and
- * hands out only fixed buffers, or in a real-time loop that may not take the
- * allocator's locks or fail on memory halfway through a unit).  Such callers
- * cannot create a ws_cache, so this call takes caller-owned K/V planes and
- * keeps its scratch (the fp32 partials of query tiles whose key range is cut
- * between CTAs, and a status word) in a file-scope device array of 48 MiB that
- * every device loading this part of the library holds until exit.
+ * for callers that must not call cudaMalloc (under a framework that owns every
+ * allocation and hands out only fixed buffers, or in a real-time loop that may
+ * not take the allocator's locks or fail on memory halfway through a unit).
+ * Such callers cannot create a ws_cache, so this call takes caller-owned K/V
+ * planes and keeps its scratch (the fp32 partials of query tiles whose key
+ * range is cut between CTAs, the merge counters and a status word) in a
+ * file-scope device array of 48 MiB that every device loading this part of the
+ * library holds until exit.
  *
  * For every head h and query row i:
  *     out[i][h] = sum_j softmax_j(q[i][h] . k_j[h] / sqrt(D)) v_j[h],  0 <= j < n_keys
@@ -287,17 +289,30 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit,
  * planes of all heads, then the V planes (the cache's per-layer layout); all
  * caller-owned device memory, 16-byte aligned.  Same arithmetic as
  * ws_unit_attention.
- * The first call on a device looks up the array's device address (with that
- * device current); make it before any stream capture.  Calls never allocate.
- * All calls share the array and it keeps the last call's contents: calls that
- * overlap on the GPU race on it, so the caller serialises them (one stream, or
- * ordering between streams).  A kernel wait that runs out leaves its status in
- * the array, which this call clears at its start and does not read back.
+ * The work runs on the current device, whose array it uses: `stream` must
+ * belong to that device (else WS_ERR_ARG).  The first call on a device (and the
+ * first after a device reset, which creates a new context) looks up the array's
+ * device address with that device current; make it before any stream capture.
+ * Calls never allocate.  All calls share the array and it keeps the last call's
+ * contents: calls that overlap on the GPU race on it, so the caller serialises
+ * them (one stream, or ordering between streams).  Each call clears the status
+ * word and the merge counters at its start.  A kernel wait that runs out (bound
+ * 2 s, or WS_WAIT_TIMEOUT_MS read at each call) leaves the output undefined and
+ * sets the status word, which ws_attention_noalloc_sync reports.
  * Errors: WS_ERR_ARG, WS_ERR_ALIGN, WS_ERR_UNSUPPORTED (head_dim other than 64 or
  * 128, or partials that would not fit the 48 MiB array), WS_ERR_CUDA.
  */
 int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query,
                          int32_t n_keys, int32_t n_heads, int32_t head_dim, cudaStream_t stream);
+
+/*
+ * ws_attention_noalloc_sync -- waits for `stream`, then reports the status word
+ * of the current device's no-alloc scratch: WS_OK, or WS_ERR_DEVICE_TIMEOUT when
+ * a bounded wait of the most recent ws_attention_noalloc call on this device
+ * ran out (the word is cleared after being read).  No counterpart in the
+ * paper.  Allocates nothing.  Errors: WS_ERR_CUDA.
+ */
+int ws_attention_noalloc_sync(cudaStream_t stream);
 
 /*
  * Unit program -- the whole device work of one streaming unit, recorded once

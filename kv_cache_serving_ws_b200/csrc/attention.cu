@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -382,17 +383,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return true;
       };
-      // O_a += P_a(g) V(g), P_a in the TMEM columns of S_a, two bf16 per column
+      // O_a += P_a(g) V(g), P_a in the TMEM columns of S_a, two bf16 per column.
+      // Rows of a partial tile past the end of its run belong to keys the query
+      // must not see (another unit's slot, stale latent rows, another session):
+      // their P is 0, but 0 * inf or 0 * NaN is NaN in the product.  The K loop
+      // stops at the 16-key step that holds the last visible key, and the rows of
+      // that step past the run's end are zeroed in shared memory first.
       auto issue_pv = [&](const TileIter& it, int a) -> bool {
         const int s = it.g & 1;
-        if (a == 0 && !warp_wait(&bars[kVFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+        const int valid = it.valid();
+        if (a == 0) {
+          if (!warp_wait(&bars[kVFull + s], ((uint32_t)it.g >> 1) & 1, guard)) return false;
+          if (valid & 15) {
+            const int r0 = valid, nz = 16 - (valid & 15);          // rows [r0, r0 + nz)
+            for (int i = lane; i < nz * S::kChunks * 8; i += 32) {
+              const int c = i / (nz * 8), rem = i - c * nz * 8;
+              uint8_t* dst = sV + s * S::kTileBytes + c * kBlockN * kRowBytes + (r0 + rem / 8) * kRowBytes +
+                             (rem & 7) * 16;
+              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+          }
+        }
         if (!warp_wait(&bars[kPFull + a], (uint32_t)it.g & 1, guard)) return false;
         if (it.first && it.n > 0 && !warp_wait(&bars[kOFree + a], (uint32_t)(it.n - 1) & 1, guard)) return false;
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_o(tmem, a);
         const uint32_t p_tmem = tmem_s(tmem, a);
+        const int steps = (valid + 15) >> 4;
 #pragma unroll
         for (int kk = 0; kk < kBlockN / 16; ++kk) {
+          if (kk >= steps) break;
           // 16 keys = 8 TMEM columns; V: 16 rows of 128 bytes, the next 64
           // head-dim columns one chunk (kBlockN rows) further
           const uint64_t db = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
@@ -732,12 +754,15 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 template <int D>
 static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
                                       int* ctas, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
+  // the shared-memory opt-in is a per-device attribute of the kernel
+  static std::atomic<bool> configured[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return cudaErrorInvalidDevice;
+  if (!configured[dev].load(std::memory_order_acquire)) {
     cudaError_t e = cudaFuncSetAttribute(unit_attention_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          Smem<D>::kAlloc);
     if (e != cudaSuccess) return e;
-    configured = true;
+    configured[dev].store(true, std::memory_order_release);
   }
   const int grid = p.dec.lanes * p.dec.lane_ctas;
   if (ctas) *ctas = grid;

@@ -11,6 +11,8 @@
 // contiguous source bytes per token and writes runs of D*2 contiguous bytes.
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "kernels.cuh"
 
 namespace ws {
@@ -81,12 +83,21 @@ __global__ void __launch_bounds__(kCopyThreads) read_kernel(const __grid_constan
 
 }  // namespace
 
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  return dev;
+}
+
 int sm_count() {
-  static int n = 0;
+  // one entry per device: a process may drive GPUs of different sizes
+  static std::atomic<int> count[kMaxDevices];
+  const int dev = current_device();
+  if (dev < 0) return 148;
+  int n = count[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    count[dev].store(n, std::memory_order_relaxed);
   }
   return n;
 }

@@ -156,6 +156,12 @@ cudaError_t launch_read(const ReadParams& p, cudaStream_t stream);
 
 cudaError_t launch_euler(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream);
 
-int sm_count();
+// Host helpers.  Kernel attributes and SM counts are per device: a process may
+// drive several GPUs, so every cached value is kept per device ordinal.
+constexpr int kMaxDevices = 64;
+int current_device();   // the current device's ordinal, or -1 (error or >= kMaxDevices)
+int sm_count();         // SMs of the current device
+// Test hook of ws_attention_noalloc (noalloc.cu): the V tile its CTAs leave out, -1 = none.
+void set_noalloc_stall(int tile);
 
 }  // namespace ws

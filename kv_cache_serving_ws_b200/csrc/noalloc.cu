@@ -2,15 +2,14 @@
 // cannot allocate device memory.
 //
 // Who needs it: code that runs where cudaMalloc is unavailable or forbidden --
-// inside a CUDA-graph capture that must not contain allocation nodes, under a
-// host framework that owns every device allocation through its own pool and
-// hands out only fixed buffers, or in a real-time loop that may not take the
+// under a host framework that owns every device allocation through its own pool
+// and hands out only fixed buffers, or in a real-time loop that may not take the
 // allocator's locks or risk an out-of-memory failure halfway through a 160 ms
 // unit.  Such a caller cannot create a ws_cache (which allocates the cache and
 // its workspace), so this entry point works on K/V planes the caller already
 // owns and keeps its own scratch -- the fp32 partials of query tiles whose key
-// range is cut between two CTAs, and the kernel's status word -- in one
-// file-scope device array instead of allocated memory.
+// range is cut between two CTAs, the in-kernel merge counters and the kernel's
+// status word -- in one file-scope device array instead of allocated memory.
 //
 // Limits and sharing: the array holds kScratchBytes (48 MiB) on every device
 // that loads this part of the library, until the process exits.  The partials
@@ -24,11 +23,18 @@
 // and the merge counters are cleared at the start of every call; the partials
 // need no clearing, because every slot a merge reads is written first by the
 // same call.
+//
+// Set-up: in host code the array's name stands for a host-side shadow, not for
+// device memory, so its device address is looked up with cudaGetSymbolAddress
+// with the device current, once per device and CUDA context (a device reset
+// creates a new context, in which the module and the array may sit elsewhere);
+// the context's unique ID tells a stale address apart.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include <nvtx3/nvToolsExt.h>
@@ -40,30 +46,71 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t(48) << 20;
 constexpr size_t kStatusBytes = 256;            // the status word, padded to keep the partials aligned
-constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
-// Device address of g_scratch per device, looked up once with that device current.
-std::mutex g_setup_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
-int scratch_address(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return WS_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (!g_scratch_addr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) return WS_ERR_CUDA;
-    g_scratch_addr[dev] = ptr;
+std::mutex g_setup_mutex;
+struct ScratchSlot {
+  unsigned long long ctx_id;   // CUDA context the address belongs to (0 = none yet)
+  void* ptr;
+};
+ScratchSlot g_slot[ws::kMaxDevices] = {};
+int g_stall_tile = -1;          // test hook (ws_debug_inject_stall with a NULL cache)
+
+// ID of the calling thread's current context, 0 if none is bound yet.
+int current_context_id(unsigned long long* id) {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  if (!get_current || !get_id) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &a, 12000, cudaEnableDefault, &qa) != cudaSuccess ||
+        qa != cudaDriverEntryPointSuccess ||
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &b, 12000, cudaEnableDefault, &qb) != cudaSuccess ||
+        qb != cudaDriverEntryPointSuccess)
+      return WS_ERR_CUDA;
+    get_current = reinterpret_cast<CtxGetCurrentFn>(a);
+    get_id = reinterpret_cast<CtxGetIdFn>(b);
   }
-  *out = g_scratch_addr[dev];
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS) return WS_ERR_CUDA;
+  *id = 0;
+  if (ctx && get_id(ctx, id) != CUDA_SUCCESS) return WS_ERR_CUDA;
   return WS_OK;
 }
 
-}  // namespace
+// Device address of g_scratch on the current device (set up on first use there).
+int scratch_address(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  unsigned long long id = 0;
+  if (current_context_id(&id) != WS_OK) return WS_ERR_CUDA;
+  ScratchSlot& slot = g_slot[dev];
+  if (id == 0 || id != slot.ctx_id || !slot.ptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return WS_ERR_CUDA;
+    }
+    if (current_context_id(&id) != WS_OK || id == 0) return WS_ERR_CUDA;
+    slot.ctx_id = id;
+    slot.ptr = ptr;
+  }
+  *out = slot.ptr;
+  return WS_OK;
+}
 
-namespace {
+uint64_t wait_bound_ns() {
+  if (const char* t = std::getenv("WS_WAIT_TIMEOUT_MS")) {
+    const long long ms = std::atoll(t);
+    if (ms > 0) return (uint64_t)ms * 1000000ull;
+  }
+  return kDefaultWaitNs;
+}
 
 int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query, int32_t n_keys,
                  int32_t n_heads, int32_t head_dim, cudaStream_t stream) {
@@ -73,6 +120,15 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
   if ((reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(kv) | reinterpret_cast<uintptr_t>(out)) & 15u)
     return WS_ERR_ALIGN;
   if ((int64_t)n_heads * 2 >= ((int64_t)1 << 31)) return WS_ERR_ARG;
+  const int dev = current_device();
+  if (dev < 0) return WS_ERR_CUDA;
+  // the scratch used is the current device's: the stream must belong to it
+  int stream_dev = -1;
+  if (cudaStreamGetDevice(stream, &stream_dev) != cudaSuccess) {
+    cudaGetLastError();
+    return WS_ERR_ARG;
+  }
+  if (stream_dev != dev) return WS_ERR_ARG;
 
   // one query unit, one run of visible keys: rows [0, n_keys) of every plane
   AttnParams p{};
@@ -96,7 +152,7 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
   if (kStatusBytes + fix_bytes + slots * slot_bytes > kScratchBytes) return WS_ERR_UNSUPPORTED;
 
   void* base = nullptr;
-  const int st = scratch_address(&base);
+  const int st = scratch_address(dev, &base);
   if (st != WS_OK) return st;
   unsigned char* b = static_cast<unsigned char*>(base);
   p.status = reinterpret_cast<int*>(b);
@@ -109,8 +165,11 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
   p.plane_v = n_heads;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   p.out = out;
-  p.timeout_ns = 2000000000ull;
-  p.debug_skip_v_tile = -1;
+  p.timeout_ns = wait_bound_ns();
+  {
+    std::lock_guard<std::mutex> lock(g_setup_mutex);
+    p.debug_skip_v_tile = g_stall_tile;
+  }
 
   CUtensorMap q_map, kv_map;
   if (encode_q_map(&q_map, q, head_dim, n_heads, n_query) != 0) return WS_ERR_CUDA;
@@ -133,10 +192,35 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
 
 }  // namespace
 
+namespace ws {
+void set_noalloc_stall(int tile) {
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  g_stall_tile = tile;
+}
+}  // namespace ws
+
 extern "C" int ws_attention_noalloc(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n_query,
                                     int32_t n_keys, int32_t n_heads, int32_t head_dim, cudaStream_t stream) {
   nvtxRangePushA("ws_attention_noalloc");   // a range for profilers (no cost without one)
   const int st = noalloc_impl(q, kv, out, n_query, n_keys, n_heads, head_dim, stream);
+  nvtxRangePop();
+  return st;
+}
+
+extern "C" int ws_attention_noalloc_sync(cudaStream_t stream) {
+  nvtxRangePushA("ws_attention_noalloc_sync");
+  int st = WS_OK;
+  int s = 0;
+  if (cudaStreamSynchronize(stream) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&s, g_scratch, sizeof(int), 0, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    st = WS_ERR_CUDA;
+  } else if (s != 0) {
+    const int zero = 0;
+    st = cudaMemcpyToSymbol(g_scratch, &zero, sizeof(int), 0, cudaMemcpyHostToDevice) == cudaSuccess
+             ? WS_ERR_DEVICE_TIMEOUT
+             : WS_ERR_CUDA;
+  }
   nvtxRangePop();
   return st;
 }

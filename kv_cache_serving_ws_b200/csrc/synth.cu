@@ -8,6 +8,7 @@
 // SplitMix64(key + (i + 1) * 0x9E3779B97F4A7C15)   (Steele, Lea, Flood 2014).
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/ws_synth.h"
@@ -16,6 +17,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kMaxTable = 8192;
+constexpr int kMaxDevices = 64;   // per-device kernel attribute flags
 
 __device__ __forceinline__ uint32_t mix_top32(uint64_t z) {
   z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -56,16 +58,17 @@ extern "C" int ws_synth_fill_normal_bf16(uint16_t* dst, int64_t n, uint64_t key,
   if (n == 0) return 0;
   if (!dst || !table_thr || !table_vals) return -1;
   const size_t smem = (sizeof(uint64_t) + sizeof(uint16_t)) * (size_t)table_len;
-  static bool configured = false;
-  if (!configured) {
+  // the shared-memory opt-in is a per-device attribute of the kernel
+  static std::atomic<bool> configured[kMaxDevices];
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -7;
+  if (!configured[dev].load(std::memory_order_acquire)) {
     if (cudaFuncSetAttribute(fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)((sizeof(uint64_t) + sizeof(uint16_t)) * kMaxTable)) != cudaSuccess)
       return -7;
-    configured = true;
+    configured[dev].store(true, std::memory_order_release);
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
   int64_t blocks = (n + kThreads - 1) / kThreads;
   if (blocks > (int64_t)sms * 4) blocks = (int64_t)sms * 4;
   fill_kernel<<<(unsigned)blocks, kThreads, smem, stream>>>(dst, n, key, index0, table_thr, table_vals,

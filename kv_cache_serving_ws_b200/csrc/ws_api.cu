@@ -537,7 +537,11 @@ int ws_cache_set_splits(ws_cache_t* h, int n_split) {
 }
 
 int ws_debug_inject_stall(ws_cache_t* h, int tile) {
-  if (!h || tile < -1) return WS_ERR_ARG;
+  if (tile < -1) return WS_ERR_ARG;
+  if (!h) {
+    set_noalloc_stall(tile);
+    return WS_OK;
+  }
   h->debug_skip_v_tile = tile;
   return WS_OK;
 }

@@ -96,6 +96,7 @@ def _declare(lib):
         "ws_plan_visible": (C.c_int, [C.POINTER(ws_cache_config), C.POINTER(i64), C.POINTER(C.c_uint8), C.c_int,
                                       i64, C.POINTER(i32), C.POINTER(i32), i32, C.POINTER(i32)]),
         "ws_attention_noalloc": (C.c_int, [_P, _P, _P, i32, i32, i32, i32, _P]),
+        "ws_attention_noalloc_sync": (C.c_int, [_P]),
         "ws_debug_inject_stall": (C.c_int, [_P, C.c_int]),
         "ws_unit_graph_create": (C.c_int, [C.POINTER(_P), _P, C.POINTER(ws_unit_io)]),
         "ws_unit_graph_launch": (C.c_int, [_P, i64, _P]),
@@ -249,7 +250,8 @@ def ws_sync(h, stream=None, check=True):
 
 
 def ws_debug_inject_stall(h, tile, check=True):
-    """Test hook: leave out one V load per CTA so the kernel's bounded wait runs out (-1 = off)."""
+    """Test hook: leave out one V load per CTA so the kernel's bounded wait runs out (-1 = off).
+    With h = None it applies to ws_attention_noalloc calls."""
     return _done(lib().ws_debug_inject_stall(h, tile), "ws_debug_inject_stall", check)
 
 
@@ -279,6 +281,11 @@ def ws_attention_noalloc(q, kv, out, n_query, n_keys, n_heads, head_dim, stream=
     """Attention over caller-owned K/V planes kv [2][H][Nk][D]; no device allocation."""
     return _done(lib().ws_attention_noalloc(_ptr(q), _ptr(kv), _ptr(out), n_query, n_keys, n_heads, head_dim,
                                             _stream(stream)), "ws_attention_noalloc", check)
+
+
+def ws_attention_noalloc_sync(stream=None, check=True):
+    """Wait for the stream; WS_ERR_DEVICE_TIMEOUT if the last no-alloc call's bounded wait ran out."""
+    return _done(lib().ws_attention_noalloc_sync(_stream(stream)), "ws_attention_noalloc_sync", check)
 
 
 def ws_pool_create(cfg: ws_cache_config, n_sessions: int, stream=None, check=True):

@@ -138,7 +138,9 @@ def test_single_unit_no_history_no_conditioning(head_dim):
     p = Pair(cfg)
     p.cond(0)
     got, want = p.attend(0, 0)
-    _check(got, want, max_tol=1e-2, mean_tol=1e-2)     # one key: out = v_new, rounded once to bf16
+    # one key: its weight is 1, so out = v_new exactly (a bf16 value times 1, rounded to bf16)
+    assert np.all(np.isfinite(got))
+    assert np.array_equal(got, want), float(np.abs(got - want).max())
     p.close()
 
 

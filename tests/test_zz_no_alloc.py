@@ -1,16 +1,30 @@
 """ws_attention_noalloc -- attention for callers that cannot allocate device memory
-(graph captures without allocation nodes, frameworks that own every allocation,
-real-time loops) -- gives the same result as ws_unit_attention on the same keys,
-for calls in a row that reuse its shared scratch array with different shapes, the
-last one long enough to merge its cut items inside the kernel.
+(frameworks that own every allocation, real-time loops that may not take the
+allocator's locks) -- gives the same result as ws_unit_attention on the same keys,
+and matches the fp64 oracle on sampled heads, for calls in a row that reuse its
+shared scratch array with different shapes, the last one long enough to merge its
+cut items inside the kernel.  A call whose bounded wait runs out is reported by
+ws_attention_noalloc_sync, and the next call is correct again.
 Kept in a file of its own, collected last."""
+import os
+
 import numpy as np
 import pytest
 import torch
 
-from gpu_util import ATOL_MAX, ATOL_MEAN, require_gpu
+from gpu_util import ATOL_MAX, ATOL_MEAN, from_dev, require_gpu
 from kv_cache_serving_ws_b200 import native as ws
 from kv_cache_serving_ws_b200 import synth
+from oracle import ws_oracle as orc
+
+
+def _oracle_heads(q, kv, heads):
+    """fp64 oracle over the caller's planes for a few heads: q [Nq][H][D], kv [2][H][Nk][D]."""
+    qb = orc.bf16_to_f64(from_dev(q))
+    kvb = from_dev(kv)
+    k = orc.bf16_to_f64(kvb[0]).transpose(1, 0, 2)        # [Nk][H][D]
+    v = orc.bf16_to_f64(kvb[1]).transpose(1, 0, 2)
+    return orc.attention_rows(qb, k, v, heads=heads)
 
 
 def _reference_and_keys(cfg, layer, seed):
@@ -66,11 +80,50 @@ def test_noalloc_matches_unit_attention_on_two_calls_in_a_row():
         out = torch.full_like(q, float("nan"))
         assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, check=False) == ws.WS_OK
         torch.cuda.synchronize()
+        assert ws.ws_attention_noalloc_sync(check=False) == ws.WS_OK
         got = out.to(torch.float64).cpu().numpy()
         want = ref.to(torch.float64).cpu().numpy()
         assert np.all(np.isfinite(got))
         d = np.abs(got - want)
         assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (cfg, float(d.max()), float(d.mean()))
+        # and against the oracle itself on two heads (first and last)
+        heads = [0, H - 1]
+        d = np.abs(got[:, heads] - _oracle_heads(q, kv, heads))
+        assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (cfg, float(d.max()), float(d.mean()))
+
+
+@pytest.mark.gpu
+def test_noalloc_reports_a_wait_that_ran_out_then_recovers():
+    """The stall hook (NULL cache: the no-alloc calls) leaves out one V load per CTA,
+    so every CTA's bounded wait (200 ms here) runs out; ws_attention_noalloc_sync
+    reports WS_ERR_DEVICE_TIMEOUT once, and the next call matches the oracle."""
+    require_gpu()
+    H, D, Nq, Nk = 4, 128, 300, 1000
+    key = lambda kind: synth.stream_key(29, kind, 0, 0)
+    q = torch.empty((Nq, H, D), dtype=torch.bfloat16, device="cuda")
+    kv = torch.empty((2, H, Nk, D), dtype=torch.bfloat16, device="cuda")
+    ws.synth_fill(q, key(synth.KIND_Q))
+    ws.synth_fill(kv, key(synth.KIND_K_NEW))
+    out = torch.empty_like(q)
+    old = os.environ.get("WS_WAIT_TIMEOUT_MS")
+    os.environ["WS_WAIT_TIMEOUT_MS"] = "200"
+    try:
+        ws.ws_debug_inject_stall(None, 0)
+        assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, check=False) == ws.WS_OK
+        assert ws.ws_attention_noalloc_sync(check=False) == ws.WS_ERR_DEVICE_TIMEOUT
+        assert ws.ws_attention_noalloc_sync(check=False) == ws.WS_OK       # read once, then cleared
+    finally:
+        ws.ws_debug_inject_stall(None, -1)
+        if old is None:
+            os.environ.pop("WS_WAIT_TIMEOUT_MS", None)
+        else:
+            os.environ["WS_WAIT_TIMEOUT_MS"] = old
+    assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, check=False) == ws.WS_OK
+    assert ws.ws_attention_noalloc_sync(check=False) == ws.WS_OK
+    got = out.to(torch.float64).cpu().numpy()
+    d = np.abs(got - _oracle_heads(q, kv, range(H)))
+    assert np.all(np.isfinite(got))
+    assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (float(d.max()), float(d.mean()))
 
 
 @pytest.mark.gpu
@@ -83,3 +136,8 @@ def test_noalloc_rejects_bad_arguments_before_any_launch():
     assert ws.ws_attention_noalloc(odd, t, t, 1, 1, 1, 64, check=False) == ws.WS_ERR_ALIGN
     # partials of 4096 query tiles x 64 heads cannot fit the 48 MiB array
     assert ws.ws_attention_noalloc(t, t, t, 4096 * 128, 1 << 20, 64, 128, check=False) == ws.WS_ERR_UNSUPPORTED
+    # a stream of another device than the current one (only with two GPUs)
+    if torch.cuda.device_count() > 1:
+        with torch.cuda.device(1):
+            other = torch.cuda.Stream()
+        assert ws.ws_attention_noalloc(t, t, t, 1, 1, 1, 64, stream=other, check=False) == ws.WS_ERR_ARG
