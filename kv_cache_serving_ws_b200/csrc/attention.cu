@@ -520,15 +520,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBlockN; ++c)
             if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
         }
-        // row max: 8 independent chains of three-input max
+        // row max: 8 independent chains, two-input max over columns 0..15, then
+        // three-input max over each further group of 16 columns
         float mx[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = __uint_as_float(sr[k]);
+        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
 #pragma unroll
-        for (int c = 8; c < kBlockN; c += 16)
+        for (int c = 16; c < kBlockN; c += 16)
 #pragma unroll
           for (int k = 0; k < 8; ++k)
             mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
+        static_assert(kBlockN % 16 == 0, "the row max takes the columns in groups of 16");
         const float m_cand =
             max3_f32(max3_f32(mx[0], mx[1], mx[2]), max3_f32(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
             p.scale_log2;
