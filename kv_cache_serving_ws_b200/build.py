@@ -24,10 +24,11 @@ FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-shared", "-c
          "--expt-relaxed-constexpr", "-I", INCLUDE]
 
 LIBS = {
-    "libws.so": ["ws_api.cu", "unit_graph.cu", "attention.cu", "copy_kernels.cu", "euler.cu", "noalloc.cu"],
+    "libws.so": ["ws_api.cu", "unit_graph.cu", "attention.cu", "attention_pair.cu", "copy_kernels.cu", "euler.cu",
+                 "noalloc.cu"],
     "libws_synth.so": ["synth.cu"],
 }
-HEADERS = ["kernels.cuh", "cache_state.cuh", "sm100.cuh", "tmem_ldst.cuh"]
+HEADERS = ["kernels.cuh", "cache_state.cuh", "sm100.cuh", "tmem_ldst.cuh", "attn_common.cuh"]
 
 
 def nvcc() -> str:

@@ -76,7 +76,8 @@ struct ws_cache {
   int* d_status = nullptr;
   int* d_fix = nullptr;               // arrival counters of the in-kernel merge of cut items
   size_t fix_bytes = 0;
-  CUtensorMap kv_map;
+  CUtensorMap kv_map;           // boxes of a whole key tile (128 rows)
+  CUtensorMap k_half_map;       // boxes of half a K tile (64 rows), for the paired kernel
   int force_lane_ctas = 0;
   int64_t slot_cap = 0;
   uint64_t timeout_ns = 2000000000ull;

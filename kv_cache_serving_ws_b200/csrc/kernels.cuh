@@ -99,17 +99,34 @@ struct AttnParams {
   KeyRuns runs;
 };
 
-// Encodes the tensor maps used by the attention kernel.  `kv` points at the
-// cache planes [planes][rows][D]; `q` at [Nq][H][D].
-int encode_kv_map(CUtensorMap* map, const void* kv, int head_dim, int64_t rows, int64_t planes);
+// Encodes the tensor maps used by the attention kernels.  `kv` points at the
+// cache planes [planes][rows][D], read in boxes of 64 columns x `box_rows` rows
+// (128 rows: a whole key tile; 64 rows: half a K tile, for the paired kernel);
+// `q` at [Nq][H][D].
+int encode_kv_map_box(CUtensorMap* map, const void* kv, int head_dim, int64_t rows, int64_t planes, int box_rows);
+inline int encode_kv_map(CUtensorMap* map, const void* kv, int head_dim, int64_t rows, int64_t planes) {
+  return encode_kv_map_box(map, kv, head_dim, rows, planes, kBlockN);
+}
 int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int n_query);
 
-cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
-                             int head_dim, int* ctas, cudaStream_t stream);
+// The attention launch: head_dim 128 runs on pairs of SMs (attention_pair.cu)
+// when the device can hold the pairs, otherwise -- and for head_dim 64 -- the
+// single-SM kernel (attention.cu).  `kv_map` has whole-tile boxes, `k_half_map`
+// boxes of 64 rows.  `p.dec` must come from decompose() with
+// attention_workers(head_dim) workers.
+cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const CUtensorMap& k_half_map,
+                             const AttnParams& p, int head_dim, int* ctas, cudaStream_t stream);
+// Workers (CTAs, or CTA pairs) of the kernel launch_attention uses for head_dim.
+int attention_workers(int head_dim);
+// CTA pairs that can be resident at once for the paired kernel (0: none).
+int pair_workers();
+cudaError_t launch_attention_pair(const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
+                                  const AttnParams& p, int* ctas, cudaStream_t stream);
 // Chooses the work decomposition of one attention call (defined in ws_api.cu):
-// the Q-block lanes together hold one CTA per SM (or `forced` CTAs per lane).
-void decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced);
-// Partial slots a decomposition needs (two per CTA).
+// the Q-block lanes together hold one worker per resident slot (`workers`), or
+// `forced` workers per lane.
+void decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int workers);
+// Partial slots a decomposition needs (two per worker).
 inline int64_t partial_slots(const Decomp& d) { return (int64_t)d.lanes * d.lane_ctas * 2; }
 
 // Merge of cut items as its own launch (when p.fixup == 0).

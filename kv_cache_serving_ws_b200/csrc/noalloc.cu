@@ -145,7 +145,7 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
 
   // scratch layout: [status | merge counters | part_ml | part_o], two partial slots per CTA
   const int n_qtiles = (n_query + kItemRows - 1) / kItemRows;
-  decompose(p.dec, n_qtiles, n_heads, p.qu.tile_start[1], 0);
+  decompose(p.dec, n_qtiles, n_heads, p.qu.tile_start[1], 0, attention_workers(head_dim));
   const size_t slots = (size_t)partial_slots(p.dec);
   const size_t slot_bytes = (size_t)kItemRows * (head_dim + 2) * sizeof(float);
   const size_t fix_bytes = ((size_t)fix_counters(1, n_qtiles, n_heads) * sizeof(int) + 255) & ~(size_t)255;
@@ -171,14 +171,15 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
     p.debug_skip_v_tile = g_stall_tile;
   }
 
-  CUtensorMap q_map, kv_map;
+  CUtensorMap q_map, kv_map, k_half_map;
   if (encode_q_map(&q_map, q, head_dim, n_heads, n_query) != 0) return WS_ERR_CUDA;
   if (encode_kv_map(&kv_map, kv, head_dim, n_keys, (int64_t)2 * n_heads) != 0) return WS_ERR_CUDA;
+  if (encode_kv_map_box(&k_half_map, kv, head_dim, n_keys, (int64_t)2 * n_heads, 64) != 0) return WS_ERR_CUDA;
 
   // the status word and the merge counters start at zero (a call that gave up may have left them set)
   if (cudaMemsetAsync(p.status, 0, kStatusBytes + fix_bytes, stream) != cudaSuccess) return WS_ERR_CUDA;
   p.fixup = use_fixup(p.dec) ? 1 : 0;
-  if (launch_attention(q_map, kv_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (launch_attention(q_map, kv_map, k_half_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
   bool any_split = false;
   for (int qt = 0; qt < n_qtiles && !any_split && !p.fixup; ++qt)
     for (int h = 0; h < n_heads && !any_split; ++h) {

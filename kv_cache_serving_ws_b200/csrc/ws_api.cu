@@ -22,8 +22,8 @@ using namespace ws;
 // per SM; the group size minimises the iterations of the busiest CTA (ties:
 // the smaller group, which re-reads K/V fewer times).  A CTA gets at least 2
 // iterations.  `forced` > 0 fixes the CTAs per lane.
-void ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced) {
-  const int sms = sm_count();
+void ws::decompose(Decomp& d, int n_qtiles, int heads, int tiles, int forced, int workers) {
+  const int sms = workers > 0 ? workers : 1;
   d.n_qtiles = n_qtiles;
   d.heads = heads;
   d.tiles = tiles;
@@ -201,9 +201,10 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   p.runs.n_runs = runs;
 
   const int n_qtiles = (h->Nq + kItemRows - 1) / kItemRows;
-  decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas);
+  const int workers = attention_workers(D);
+  decompose(p.dec, n_qtiles, H, tiles, h->force_lane_ctas, workers);
   while (partial_slots(p.dec) > h->slot_cap && p.dec.lane_ctas > 1)
-    decompose(p.dec, n_qtiles, H, tiles, std::max(1, p.dec.lane_ctas / 2));
+    decompose(p.dec, n_qtiles, H, tiles, std::max(1, p.dec.lane_ctas / 2), workers);
   if (partial_slots(p.dec) > h->slot_cap) return WS_ERR_UNSUPPORTED;
   p.fixup = use_fixup(p.dec) ? 1 : 0;
   bool any_split = false;
@@ -255,7 +256,7 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_attn.next() : nullptr;
   if (ev) cudaEventRecord(ev[0], stream);
   int ctas = 0;
-  if (launch_attention(q_map, h->kv_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (launch_attention(q_map, h->kv_map, h->k_half_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
   if (any_split) {
     ev = h->profiling && !h->capturing ? h->ev_comb.next() : nullptr;
@@ -392,7 +393,9 @@ int ws_pool_create(ws_cache_t** out, const ws_cache_config* cfg, int32_t n_sessi
                       cudaMemsetAsync(h->d_status, 0, sizeof(int), stream) != cudaSuccess ||
                       cudaMemsetAsync(h->d_fix, 0, h->fix_bytes, stream) != cudaSuccess))
     st = WS_ERR_CUDA;
-  if (st == WS_OK && encode_kv_map(&h->kv_map, h->kv, D, rows, (int64_t)L * 2 * H) != 0) st = WS_ERR_CUDA;
+  if (st == WS_OK && (encode_kv_map(&h->kv_map, h->kv, D, rows, (int64_t)L * 2 * H) != 0 ||
+                      encode_kv_map_box(&h->k_half_map, h->kv, D, rows, (int64_t)L * 2 * H, 64) != 0))
+    st = WS_ERR_CUDA;
   if (st != WS_OK) {
     cudaGetLastError();
     free_all(h);

@@ -52,7 +52,9 @@ def test_inject_hook_validates_its_argument():
     require_gpu()
     _, h = ws.ws_cache_create(ws.make_config(1, 1, 64, 4, 0, 0, 0))
     assert ws.ws_debug_inject_stall(h, -2, check=False) == ws.WS_ERR_ARG
-    assert ws.ws_debug_inject_stall(None, 0, check=False) == ws.WS_ERR_ARG
+    # a NULL cache addresses the no-alloc calls' hook: -1 (off) is accepted, -2 is not
+    assert ws.ws_debug_inject_stall(None, -2, check=False) == ws.WS_ERR_ARG
+    assert ws.ws_debug_inject_stall(None, -1, check=False) == ws.WS_OK
     ws.ws_cache_destroy(h)
 
 
