@@ -33,7 +33,8 @@ METRIC = "block-causal unit-attention TFLOP/s & ms per 640×368 unit on 1 B200 (
 UNIT = "TFLOP/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "unit_attention_traffic.txt")
-KERNEL_SOURCES = ["kv_cache_serving_ws_b200/csrc/attention.cu", "kv_cache_serving_ws_b200/csrc/sm100.cuh",
+KERNEL_SOURCES = ["kv_cache_serving_ws_b200/csrc/attention.cu", "kv_cache_serving_ws_b200/csrc/attention_pair.cu",
+                  "kv_cache_serving_ws_b200/csrc/attn_common.cuh", "kv_cache_serving_ws_b200/csrc/sm100.cuh",
                   "kv_cache_serving_ws_b200/csrc/kernels.cuh", "kv_cache_serving_ws_b200/csrc/tmem_ldst.cuh"]
 
 
@@ -463,6 +464,41 @@ def oracle_sample(target_s: float, max_rows=None):
             "seconds": round(dt, 2)}
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def oracle_config(w, heads: int, rows=None):
+    """The fp64 oracle over `heads` heads (all query rows unless `rows`) of one attention
+    call of workload w, timed on the host cores; the whole call is extrapolated from the
+    sample by heads and rows (factor 1 = timed in full).  Input generation is not timed."""
+    sys.path.insert(0, os.path.join(ROOT, "tests"))
+    from oracle_side import oracle_cache
+    cache, q, kn, vn = oracle_cache(w, 0, list(range(heads)))
+    rows = w.n_query if rows is None else rows
+    t0 = time.perf_counter()
+    st, _ = cache.unit_attention(0, w.unit, q, kn, vn, rows=list(range(rows)), heads=list(range(heads)))
+    dt = time.perf_counter() - t0
+    assert st == 0
+    factor = (w.n_heads / heads) * (w.n_query / rows)
+    flops = 4.0 * rows * heads * w.n_keys * w.head_dim
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+    return {"kind": "oracle", "value": round(flops / dt / 1e12, 6), "unit": UNIT,
+            "ms_per_call": round(dt * factor * 1e3, 1), "extrapolated_x": round(factor, 2),
+            "sample": f"{heads} of {w.n_heads} heads x {rows} of {w.n_query} query rows in {dt:.2f} s",
+            "cores": int(cores), "cpu": cpu_model()}
+
+
 def run_reference(args):
     rank, _, world = dist_env()
     if rank != 0:
@@ -824,16 +860,23 @@ def run_configs(args):
         io_bytes = 4 * w.n_query * w.n_heads * w.head_dim * 2
         t_compute = flops / (pk["bf16"] * 1e12) * 1e3
         t_memory = (kv_bytes + io_bytes) / (pk["hbm"] * 1e9) * 1e3
-        print(json.dumps({"mode": "configs", "workload": w.name, "calls": args.calls, "l2": "flushed before each call",
-                          "ms_median": round(med, 4), "ms_min": round(mn, 4),
-                          "TFLOP/s": round(flops / med / 1e9, 1),
-                          "frac_of_burst_bf16": round(flops / med / 1e9 / pk["bf16"], 4),
-                          "bytes": kv_bytes + io_bytes, "GB/s": round((kv_bytes + io_bytes) / med / 1e6, 1),
-                          "frac_of_measured_hbm": round((kv_bytes + io_bytes) / med / 1e6 / pk["hbm"], 4),
-                          "roofline_ms": round(max(t_compute, t_memory), 4),
-                          "bound": "tensor" if t_compute >= t_memory else "hbm",
-                          "status": ws.status_string(st)}), flush=True)
+        line = {"mode": "configs", "workload": w.name, "calls": args.calls, "l2": "flushed before each call",
+                "ms_median": round(med, 4), "ms_min": round(mn, 4),
+                "TFLOP/s": round(flops / med / 1e9, 1),
+                "frac_of_burst_bf16": round(flops / med / 1e9 / pk["bf16"], 4),
+                "bytes": kv_bytes + io_bytes, "GB/s": round((kv_bytes + io_bytes) / med / 1e6, 1),
+                "frac_of_measured_hbm": round((kv_bytes + io_bytes) / med / 1e6 / pk["hbm"], 4),
+                "roofline_ms": round(max(t_compute, t_memory), 4),
+                "bound": "tensor" if t_compute >= t_memory else "hbm",
+                "status": ws.status_string(st)}
         g.close()
+        if not args.no_cpu_baseline:
+            # the oracle beside it: in full for the tiny and 192x336 cases, four heads
+            # (all rows) at 640x368 and one head of the 128-unit ring, extrapolated
+            heads = {TINY.name: TINY.n_heads, V01.name: V01.n_heads, V02.name: 4, RING.name: 1}[w.name]
+            line["cpu_baseline"] = oracle_config(w, heads)
+            line["cpu_baseline"]["gpu_speedup"] = round(line["cpu_baseline"]["ms_per_call"] / med, 1)
+        print(json.dumps(line), flush=True)
         if args.library:
             for name, res in library_attention(w, args.calls, flush):
                 line = {"mode": "configs", "impl": "library:" + name, "workload": w.name, "calls": args.calls,

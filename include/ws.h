@@ -65,7 +65,8 @@ enum {
   WS_ERR_NOT_READY = -6,       /* the unit (or its latent segment) was never written */
   WS_ERR_CUDA = -7,            /* a CUDA runtime call or launch failed */
   WS_ERR_DEVICE_TIMEOUT = -8,  /* a kernel's bounded wait ran out (reported by ws_sync) */
-  WS_ERR_UNSUPPORTED = -9      /* valid request outside what this build supports (e.g. D not 64/128) */
+  WS_ERR_UNSUPPORTED = -9,     /* valid request outside what this build supports (e.g. D not 64/128) */
+  WS_ERR_DEVICE_CHECK = -10    /* a device-side index check failed (libws_debug.so only; ws_sync) */
 };
 
 /* Segments of a unit slot: the thinker's conditioning tokens, then the unit's latent tokens. */
@@ -215,7 +216,11 @@ int ws_cache_set_splits(ws_cache_t* h, int n_split);
 /*
  * ws_sync -- synchronise `stream`, then read and clear the device status word.
  * Returns WS_ERR_DEVICE_TIMEOUT if a kernel gave up a bounded wait since the
- * last ws_sync, WS_ERR_CUDA on a CUDA error, else WS_OK.
+ * last ws_sync, WS_ERR_DEVICE_CHECK if a device-side index check failed (only
+ * the checked build, libws_debug.so, has these checks: every computed cache row,
+ * output row, partial slot and merge counter is tested against its buffer's
+ * bounds, and a failing access is skipped instead of made), WS_ERR_CUDA on a
+ * CUDA error, else WS_OK.
  */
 int ws_sync(ws_cache_t* h, cudaStream_t stream);
 
@@ -240,6 +245,7 @@ typedef struct {
   int32_t last_n_split;        /* CTAs per query-pair lane of the last attention call */
   int32_t last_ctas;           /* CTAs of the last attention launch */
   int64_t last_keys;           /* visible keys of the last attention call */
+  int32_t last_kernel;         /* kernel of the last attention launch: 1 single-SM, 2 pairs of SMs */
 } ws_profile;
 
 int ws_profile_enable(ws_cache_t* h, int enable);   /* enabling resets the totals */

@@ -37,6 +37,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
+#include <string>
 
 #include "attn_common.cuh"
 #include "kernels.cuh"
@@ -174,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = g & 1;
         const uint32_t use = (uint32_t)g >> 1;
         const int row0 = it.row0();
+        it.check_run(p);
         if (use > 0 && !wait_phase(&bars[kKEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars[kKFull + s], S::kTileBytes);
         for (int c = 0; c < S::kChunks; ++c)
@@ -363,20 +365,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c = 0; c < kBlockN; ++c)
             if (c >= valid) sr[c] = __float_as_uint(-INFINITY);
         }
-        // row max: 8 independent chains, two-input max over columns 0..15, then
-        // three-input max over each further group of 16 columns
-        float mx[8];
+        // row max: 4 independent chains of three-input max (8 chains need more
+        // registers than the 168 a thread has here)
+        float mx[4];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mx[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[8 + k]));
+        for (int k = 0; k < 4; ++k) mx[k] = fmaxf(__uint_as_float(sr[k]), __uint_as_float(sr[4 + k]));
 #pragma unroll
-        for (int c = 16; c < kBlockN; c += 16)
+        for (int c = 8; c < kBlockN; c += 8)
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 8 + k]));
-        static_assert(kBlockN % 16 == 0, "the row max takes the columns in groups of 16");
-        const float m_cand =
-            max3_f32(max3_f32(mx[0], mx[1], mx[2]), max3_f32(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])) *
-            p.scale_log2;
+          for (int k = 0; k < 4; ++k)
+            mx[k] = max3_f32(mx[k], __uint_as_float(sr[c + k]), __uint_as_float(sr[c + 4 + k]));
+        static_assert(kBlockN % 8 == 0, "the row max takes the columns in groups of 8");
+        const float m_cand = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * p.scale_log2;
         // Move the reference max when P would exceed 2^8, for a new item, or to
         // the row max when this row's sum triggered the recomputation.
         move = it.first || m_cand > m_ref + 8.f || (hot && m_cand > m_ref);
@@ -432,14 +432,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         int lane_i, c_first, pieces, end0;
         item_span(d, p.qu, it.j, it.qt(), it.h, lane_i, c_first, pieces, end0);
         const float inv = 1.f / l_sum;
-        const bool in_unit = r_unit < p.qu.rows;
+        const bool in_unit =
+            r_unit < p.qu.rows && index_ok((int64_t)it.j * p.qu.rows + r_unit < p.out_rows, p.status);
         uint16_t* dst = p.out + ((size_t)(it.j * p.qu.rows + r_unit) * p.n_heads + it.h) * D;
         size_t prow = 0;
+        bool part_ok = true;
         if (pieces > 1) {
           // this CTA's first item takes slot (cta, 0), any later one slot (cta, 1)
           const size_t slot = partial_slot(d, rg.lane, rg.idx, it.n == 0 ? 0 : 1);
           prow = slot * kItemRows + (size_t)(a * kBlockM + row);
-          *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
+          part_ok = index_ok(slot < (size_t)p.part_slots, p.status);
+          if (part_ok) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
         }
         // O in 32-column chunks: bf16 output of a whole item, fp32 partial otherwise
 #pragma unroll 1
@@ -458,7 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *reinterpret_cast<uint4*>(dst + c + k) = v;
               }
             }
-          } else {
+          } else if (part_ok) {
             float* po = p.part_o + prow * D + c;
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
@@ -474,9 +477,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           __threadfence();
           __syncwarp();
           const size_t ci =
-              ((((size_t)it.j * d.n_qtiles + it.qt()) * p.n_heads + it.h) * kQTiles + a) * 4 + (warp & 3);
+              ((((size_t)it.j * d.n_qtiles + it.qt()) * p.n_heads + it.h) * kQTiles + a) * kFixPerTile + (warp & 3);
           int last = 0;
-          if (lane == 0) last = atomicAdd(p.fix_count + ci, 1) == pieces - 1;
+          if (lane == 0 && index_ok(ci < (size_t)p.fix_slots && part_ok, p.status))
+            last = atomicAdd(p.fix_count + ci, 1) == pieces - 1;
           last = __shfl_sync(0xffffffffu, last, 0);
           if (last) {
             if (lane == 0) p.fix_count[ci] = 0;
@@ -516,6 +520,10 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Attn
   int lane_i, c_first, pieces, end0;
   item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
   if (pieces == 1) return;                       // written directly by its CTA
+  if (!index_ok(partial_slot(p.dec, lane_i, c_first + pieces - 1, 0) < (size_t)p.part_slots &&
+                    (int64_t)row < p.out_rows,
+                p.status))
+    return;
   // piece k was written by CTA c_first + k: its last item for k = 0 (unless
   // the item starts exactly at that CTA's range), its first item otherwise
   float m_all = -INFINITY;
@@ -623,17 +631,21 @@ static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMa
 }
 
 namespace {
-// WS_ATTENTION_SINGLE_SM=1 keeps head_dim 128 on the single-SM kernel (for comparisons).
+// head_dim 128 runs on the single-SM kernel, which is the faster of the two on
+// every measured shape; WS_ATTENTION_KERNEL=pair (read once per process) selects
+// the kernel on pairs of SMs (attention_pair.cu) instead, where the device can
+// hold its clusters.
 bool use_pair_kernel(int head_dim) {
-  static const bool single = [] {
-    const char* e = std::getenv("WS_ATTENTION_SINGLE_SM");
-    return e && e[0] == '1';
+  static const bool pair = [] {
+    const char* e = std::getenv("WS_ATTENTION_KERNEL");
+    return e && std::string(e) == "pair";
   }();
-  return head_dim == 128 && !single && pair_workers() > 0;
+  return head_dim == 128 && pair && pair_workers() > 0;
 }
 }  // namespace
 
 int attention_workers(int head_dim) { return use_pair_kernel(head_dim) ? pair_workers() : sm_count(); }
+bool attention_uses_pairs(int head_dim) { return use_pair_kernel(head_dim); }
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const CUtensorMap& k_half_map,
                              const AttnParams& p, int head_dim, int* ctas, cudaStream_t stream) {

@@ -22,7 +22,7 @@
 // core computes S(g+1) and S(g+2) while the softmax works on S(g), so the
 // softmax is no longer waiting on the products of its own previous tile.
 //
-// Roles in each CTA (224 threads):
+// Roles in each CTA (256 threads):
 //   warps 0-3  softmax of this CTA's 128 rows (one row per thread = TMEM lane):
 //              fp32 online softmax in base 2 with a lazily moved reference max,
 //              P rounded to bf16 into the TMEM columns of its own S; the
@@ -31,16 +31,25 @@
 //              K tile (four stages);
 //   warp 5     TMA producer of this CTA's half of every V tile (three stages);
 //              in a partial tile it zeroes the value rows past the run's end;
-//   warp 6     leader: MMA issuer; both CTAs: TMEM allocation.
-// Order of the products: S(0), S(1), S(2), then per tile PV(g), S(g+3).
+//   warp 6     leader: issues every P.V product; both CTAs: TMEM allocation;
+//   warp 7     leader: issues every S product.
+// Issuing one M = 256 product takes the issuing warp longer than the tensor core
+// takes to run it, so the two kinds of product come from two warps.  S(g+3)
+// overwrites the S buffer whose P the product P.V(g) reads: the S warp waits for
+// that product's completion (a commit) before it issues S(g+3).
 // TMEM (each SM): O [0,128), S buffer b at [128 + 128 b, 256 + 128 b).
 //
 // Cross-CTA signalling: copies of both CTAs complete on the leader's "full"
 // barriers (cta_group::2 TMA with the leader's barrier), the leader's commits
 // arrive on both CTAs' barriers (one commit per barrier, the peer's addressed
 // through the shared::cluster window), and the peer's softmax and V producer
-// arrive remotely on the leader's barriers.  Every wait is bounded; a wait that
-// runs out raises the abort flag of both CTAs and stores a status for ws_sync.
+// arrive remotely on the leader's barriers.  Those remote arrivals are plain
+// counts: P and O live in TMEM, ordered by tcgen05.wait and the tcgen05
+// thread-sync fences, and V halves by their transaction bytes -- except a
+// partial V tile whose rows the peer zeroed with ordinary stores, which it
+// reports with a release at cluster scope that the leader acquires.  Every wait
+// is bounded; a wait that runs out raises the abort flag of both CTAs and
+// stores a status for ws_sync.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -64,8 +73,9 @@ constexpr int kVStages = 3;
 constexpr int kSoftWarps = 4;
 constexpr int kKWarp = 4;
 constexpr int kVWarp = 5;
-constexpr int kMmaWarpP = 6;
-constexpr int kPairThreads = 32 * 7;
+constexpr int kPvWarp = 6;
+constexpr int kSWarp = 7;
+constexpr int kPairThreads = 32 * 8;
 constexpr int kRowB = 128;          // one 128-byte swizzle row = 64 bf16
 
 enum PBar : int {
@@ -81,8 +91,10 @@ enum PBar : int {
   pPVDone = 27,     // +2  both: P.V of tiles with this parity
   pOFull = 29,      //     both: O of an item complete
   pOFree = 30,      //     leader: 8 warps have read O
-  pMmaDone = 31,    //     leader
-  pNumBars = 32
+  pPvDone = 31,     //     leader: every P.V product complete (leaving)
+  pSBufFree = 32,   // +3  leader: P.V of the buffer's tile complete
+  pSDone = 35,      //     leader: every S product complete (leaving)
+  pNumBars = 36
 };
 
 struct PSmem {
@@ -118,10 +130,11 @@ struct PairGuard {
   uint64_t timeout_ns;
 };
 
-__device__ __noinline__ bool pair_wait_slow(uint64_t* bar, uint32_t parity, const PairGuard& g) {
+// Waits acquire at CTA scope, except pair_wait_cluster (see the signalling notes).
+__device__ __noinline__ bool pair_wait_slow(uint64_t* bar, uint32_t parity, const PairGuard& g, bool cluster) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0; it < (1u << 28); ++it) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
+    if (cluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 31u) {
       if (*g.abort_flag) return false;
       if (global_timer_ns() - t0 > g.timeout_ns) break;
@@ -133,11 +146,34 @@ __device__ __noinline__ bool pair_wait_slow(uint64_t* bar, uint32_t parity, cons
   return false;
 }
 __device__ __forceinline__ bool pair_wait(uint64_t* bar, uint32_t parity, const PairGuard& g) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return pair_wait_slow(bar, parity, g, false);
+}
+__device__ __forceinline__ bool pair_wait_cluster(uint64_t* bar, uint32_t parity, const PairGuard& g) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
-  return pair_wait_slow(bar, parity, g);
+  return pair_wait_slow(bar, parity, g, true);
 }
 __device__ __forceinline__ bool pair_warp_wait(uint64_t* bar, uint32_t parity, const PairGuard& g) {
   return __all_sync(0xffffffffu, pair_wait(bar, parity, g));
+}
+__device__ __forceinline__ bool pair_warp_wait_cluster(uint64_t* bar, uint32_t parity, const PairGuard& g) {
+  return __all_sync(0xffffffffu, pair_wait_cluster(bar, parity, g));
+}
+
+// P = 2^(s * log2(e)/sqrt(D) - m) of one row's 128 S values, packed to bf16 pairs in pk,
+// the fp32 sums in four chains of pairs.
+__device__ __forceinline__ void softmax_pairs(const uint32_t (&sr)[kBlockN], uint64_t scale2, uint64_t negm2,
+                                              uint64_t (&rs2)[4], uint32_t (&pk)[kBlockN / 2]) {
+#pragma unroll
+  for (int c = 0; c < kBlockN / 2; ++c) {
+    const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
+    float x0, x1;
+    f32x2_split(x, x0, x1);
+    const float e0 = ex2_approx(x0);
+    const float e1 = ex2_approx(x1);
+    rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
+    pk[c] = pack_bf16x2(e0, e1);
+  }
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
@@ -185,7 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == kMmaWarpP) {
+  if (warp == kPvWarp) {
     tmem_alloc_pair(tmem_slot, 512);
     tmem_relinquish_pair();
   }
@@ -229,6 +265,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                              it.j * p.qu.rows + it.qt() * kItemRows + (int)rank * kBlockM);
           issued_q[qb] = it.n;
         }
+        it.check_run(p);
         if (g >= kKStages && !pair_wait(&bars[pKEmpty + kr.idx], kr.ph ^ 1u, guard)) {
           ok = false;
           break;
@@ -276,7 +313,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (lane == 0) {
           if (leader) mbar_arrive_expect_tx(&bars[pVFull + vr.idx], 2 * S::kVBytes);
           tma_load_3d_pair(dst, &v_map, lead_bar(pVFull + vr.idx), (int)rank * 64, it.row0(), p.plane_v + it.h);
-          if (!leader) mbar_arrive_cluster(lead_bar(pVFull + vr.idx));
+          if (!leader) mbar_arrive_cluster_relaxed(lead_bar(pVFull + vr.idx));
         }
       } else {
         // Rows of this tile past the end of the run belong to keys the query must
@@ -310,7 +347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
       vr.next();
     }
-    if (!ok || *abort_flag) {
+    // one decision for the whole warp (lanes may read the abort flag at different times)
+    if (__any_sync(0xffffffffu, !ok || *abort_flag)) {
       if (lane == 0) {
         for (int i = 0; i < kVStages; ++i)
           if (issued_local[i]) drain_wait(&bars[pVLocal + i], ((local_ph >> i) & 1u) ^ 1u, p.timeout_ns);
@@ -318,79 +356,84 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       }
       __syncwarp();
     }
-  } else if (warp == kMmaWarpP) {
+  } else if (warp == kPvWarp || warp == kSWarp) {
     if (leader) {
-      // ---------------------------------------------------- MMA issuer
-      constexpr uint32_t idesc_s = umma_idesc_bf16_f32(256, kBlockN, false, false);
-      constexpr uint32_t idesc_o = umma_idesc_bf16_f32(256, kPD, false, true);
+      // ---------------------------------------------------- MMA issuers
       const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK), v_base = smem_u32(sV);
-      TileIter its, itp;
-      its.init(d, p.qu, p.runs, rg);
-      itp = its;
-      RingPos<kSBufs> sb_s, sb_p;
-      RingPos<kKStages> kr;
-      RingPos<kVStages> vr;
       auto commit_both = [&](int i) {
         if (elect_one()) {
           umma_commit_pair(lead_bar(i));
           umma_commit_pair(peer_bar(i));
         }
       };
-      // S(g) = Q K(g)^T into S buffer sb_s
-      auto issue_s = [&]() -> bool {
-        const int qb = its.n & 1;
-        if (its.first && !pair_warp_wait(&bars[pQFull + qb], (uint32_t)(its.n >> 1) & 1, guard)) return false;
-        if (!pair_warp_wait(&bars[pKFull + kr.idx], kr.ph, guard)) return false;
-        tc_fence_after_sync();
-        const uint32_t d_tmem = tmem + 128u + 128u * (uint32_t)sb_s.idx;
-#pragma unroll
-        for (int kk = 0; kk < kPD / 16; ++kk) {
-          const uint32_t qoff = (uint32_t)((kk >> 2) * 128 * kRowB + (kk & 3) * 32);
-          const uint32_t koff = (uint32_t)((kk >> 2) * 64 * kRowB + (kk & 3) * 32);
-          const uint64_t da = umma_smem_desc_sw128(q_base + qb * S::kQBytes + qoff, 16, 1024);
-          const uint64_t db = umma_smem_desc_sw128(k_base + kr.idx * S::kKBytes + koff, 16, 1024);
-          if (elect_one()) umma_bf16_ss_pair(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
-        }
-        commit_both(pSFull + sb_s.idx);
-        commit_both(pKEmpty + kr.idx);
-        if (its.last) commit_both(pQEmpty + qb);
-        sb_s.next();
-        kr.next();
-        its.next(p.qu, p.runs);
-        return true;
-      };
-      // O += P(g) V(g), P in the TMEM columns of its S buffer, two bf16 per column
-      auto issue_pv = [&](int g) -> bool {
-        if (!pair_warp_wait(&bars[pVFull + vr.idx], vr.ph, guard)) return false;
-        if (!pair_warp_wait(&bars[pPFull + sb_p.idx], sb_p.ph, guard)) return false;
-        if (itp.first && itp.n > 0 && !pair_warp_wait(&bars[pOFree], (uint32_t)(itp.n - 1) & 1, guard)) return false;
-        tc_fence_after_sync();
-        const uint32_t p_tmem = tmem + 128u + 128u * (uint32_t)sb_p.idx;
-        const int steps = (itp.valid() + 15) >> 4;
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          if (kk >= steps) break;
-          // 16 keys = 8 TMEM columns of P; V: 16 rows of 128 bytes
-          const uint64_t db = umma_smem_desc_sw128(v_base + vr.idx * S::kVBytes + kk * 16 * kRowB, 128 * kRowB, 1024);
-          if (elect_one()) umma_bf16_ts_pair(tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!itp.first || kk > 0) ? 1u : 0u);
-        }
-        commit_both(pVEmpty + vr.idx);
-        commit_both(pPVDone + (g & 1));
-        if (itp.last) commit_both(pOFull);
-        sb_p.next();
-        vr.next();
-        itp.next(p.qu, p.runs);
-        return true;
-      };
+      TileIter it;
+      it.init(d, p.qu, p.runs, rg);
+      RingPos<kSBufs> sb;
       bool ok = true;
-      const int pre = len < kSBufs ? len : kSBufs;
-      for (int i = 0; ok && i < pre; ++i) ok = issue_s();
-      for (int g = 0; ok && g < len; ++g) {
-        ok = issue_pv(g);
-        if (ok && g + kSBufs < len) ok = issue_s();
+      if (warp == kSWarp) {
+        // S(g) = Q K(g)^T into S buffer g mod 3, once P.V(g-3) has read that buffer's P
+        constexpr uint32_t idesc_s = umma_idesc_bf16_f32(256, kBlockN, false, false);
+        RingPos<kKStages> kr;
+        for (int g = 0; ok && g < len; ++g, it.next(p.qu, p.runs)) {
+          const int qb = it.n & 1;
+          if (g >= kSBufs && !pair_warp_wait(&bars[pSBufFree + sb.idx], sb.ph ^ 1u, guard)) ok = false;
+          if (ok && it.first && !pair_warp_wait(&bars[pQFull + qb], (uint32_t)(it.n >> 1) & 1, guard)) ok = false;
+          if (ok && !pair_warp_wait(&bars[pKFull + kr.idx], kr.ph, guard)) ok = false;
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t d_tmem = tmem + 128u + 128u * (uint32_t)sb.idx;
+          // descriptors of the chunk starts; a K step adds its byte offset / 16 to the address field
+          const uint64_t da0 = umma_smem_desc_sw128(q_base + qb * S::kQBytes, 16, 1024);
+          const uint64_t db0 = umma_smem_desc_sw128(k_base + kr.idx * S::kKBytes, 16, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kPD / 16; ++kk) {
+            const uint32_t qoff = (uint32_t)((kk >> 2) * 128 * kRowB + (kk & 3) * 32);
+            const uint32_t koff = (uint32_t)((kk >> 2) * 64 * kRowB + (kk & 3) * 32);
+            const uint64_t da = da0 + (uint64_t)(qoff >> 4);
+            const uint64_t db = db0 + (uint64_t)(koff >> 4);
+            if (elect_one()) umma_bf16_ss_pair(d_tmem, da, db, idesc_s, kk > 0 ? 1u : 0u);
+          }
+          commit_both(pSFull + sb.idx);
+          commit_both(pKEmpty + kr.idx);
+          if (it.last) commit_both(pQEmpty + qb);
+          sb.next();
+          kr.next();
+        }
+        if (elect_one()) umma_commit_pair(lead_bar(pSDone));
+        drain_wait(&bars[pSDone], 0, p.timeout_ns);
+      } else {
+        // O += P(g) V(g), P in the TMEM columns of its S buffer, two bf16 per column
+        constexpr uint32_t idesc_o = umma_idesc_bf16_f32(256, kPD, false, true);
+        RingPos<kVStages> vr;
+        for (int g = 0; ok && g < len; ++g, it.next(p.qu, p.runs)) {
+          const int valid = it.valid();
+          // a partial tile's V rows were zeroed by ordinary stores, in the peer too
+          if ((valid & 15) != 0) ok = pair_warp_wait_cluster(&bars[pVFull + vr.idx], vr.ph, guard);
+          else ok = pair_warp_wait(&bars[pVFull + vr.idx], vr.ph, guard);
+          if (ok && !pair_warp_wait(&bars[pPFull + sb.idx], sb.ph, guard)) ok = false;
+          if (ok && it.first && it.n > 0 && !pair_warp_wait(&bars[pOFree], (uint32_t)(it.n - 1) & 1, guard)) ok = false;
+          if (!ok) break;
+          tc_fence_after_sync();
+          const uint32_t p_tmem = tmem + 128u + 128u * (uint32_t)sb.idx;
+          const int steps = (valid + 15) >> 4;
+          const uint64_t dv0 = umma_smem_desc_sw128(v_base + vr.idx * S::kVBytes, 128 * kRowB, 1024);
+#pragma unroll
+          for (int kk = 0; kk < kBlockN / 16; ++kk) {
+            if (kk >= steps) break;
+            // 16 keys = 8 TMEM columns of P; V: 16 rows of 128 bytes
+            const uint64_t db = dv0 + (uint64_t)((kk * 16 * kRowB) >> 4);
+            if (elect_one()) umma_bf16_ts_pair(tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
+          }
+          if (elect_one()) umma_commit_pair(lead_bar(pSBufFree + sb.idx));
+          commit_both(pVEmpty + vr.idx);
+          commit_both(pPVDone + (g & 1));
+          if (it.last) commit_both(pOFull);
+          sb.next();
+          vr.next();
+        }
+        if (elect_one()) umma_commit_pair(lead_bar(pPvDone));
+        drain_wait(&bars[pPvDone], 0, p.timeout_ns);
       }
-      if (elect_one()) umma_commit_pair(lead_bar(pMmaDone));
-      drain_wait(&bars[pMmaDone], 0, p.timeout_ns);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -437,16 +480,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint64_t negm2 = f32x2(-m_ref, -m_ref);
 #pragma unroll
         for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kBlockN / 2; ++c) {
-          const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
-          float x0, x1;
-          f32x2_split(x, x0, x1);
-          const float e0 = ex2_approx(x0);
-          const float e1 = ex2_approx(x1);
-          rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
-          pk[c] = pack_bf16x2(e0, e1);
-        }
+        softmax_pairs(sr, scale2, negm2, rs2, pk);
         float rs[8];
         f32x2_split(rs2[0], rs[0], rs[1]);
         f32x2_split(rs2[1], rs[2], rs[3]);
@@ -486,16 +520,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint64_t negm2 = f32x2(-m_ref, -m_ref);
 #pragma unroll
         for (int k = 0; k < 4; ++k) rs2[k] = f32x2(0.f, 0.f);
-#pragma unroll
-        for (int c = 0; c < kBlockN / 2; ++c) {
-          const uint64_t x = fma_f32x2(f32x2(__uint_as_float(sr[2 * c]), __uint_as_float(sr[2 * c + 1])), scale2, negm2);
-          float x0, x1;
-          f32x2_split(x, x0, x1);
-          const float e0 = ex2_approx(x0);
-          const float e1 = ex2_approx(x1);
-          rs2[c & 3] = add_f32x2(rs2[c & 3], f32x2(e0, e1));
-          pk[c] = pack_bf16x2(e0, e1);
-        }
+        softmax_pairs(sr, scale2, negm2, rs2, pk);
       }
       {
         float rs[8];
@@ -526,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (leader)
           mbar_arrive(&bars[pPFull + sb.idx]);
         else
-          mbar_arrive_cluster(lead_bar(pPFull + sb.idx));
+          mbar_arrive_cluster_relaxed(lead_bar(pPFull + sb.idx));
       }
       sb.next();
 
@@ -539,14 +564,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         int lane_i, c_first, pieces, end0;
         item_span(d, p.qu, it.j, it.qt(), it.h, lane_i, c_first, pieces, end0);
         const float inv = 1.f / l_sum;
-        const bool in_unit = r_unit < p.qu.rows;
+        const bool in_unit =
+            r_unit < p.qu.rows && index_ok((int64_t)it.j * p.qu.rows + r_unit < p.out_rows, p.status);
         uint16_t* dst = p.out + ((size_t)(it.j * p.qu.rows + r_unit) * p.n_heads + it.h) * kPD;
         size_t prow = 0;
+        bool part_ok = true;
         if (pieces > 1) {
           // this worker's first item takes slot (worker, 0), any later one slot (worker, 1)
           const size_t slot = partial_slot(d, rg.lane, rg.idx, it.n == 0 ? 0 : 1);
           prow = slot * kItemRows + (size_t)(a * kBlockM + row);
-          *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
+          part_ok = index_ok(slot < (size_t)p.part_slots, p.status);
+          if (part_ok) *reinterpret_cast<float2*>(p.part_ml + prow * 2) = make_float2(m_ref, l_sum);
         }
 #pragma unroll 1
         for (int c = 0; c < kPD; c += 32) {
@@ -564,7 +592,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
                 *reinterpret_cast<uint4*>(dst + c + k) = v;
               }
             }
-          } else {
+          } else if (part_ok) {
             float* po = p.part_o + prow * kPD + c;
 #pragma unroll
             for (int k = 0; k < 32; k += 4)
@@ -577,7 +605,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           if (leader)
             mbar_arrive(&bars[pOFree]);
           else
-            mbar_arrive_cluster(lead_bar(pOFree));
+            mbar_arrive_cluster_relaxed(lead_bar(pOFree));
         }
         if (pieces > 1 && p.fixup) {
           // Stream-K fix-up: the last piece of the item to arrive merges these 32
@@ -585,9 +613,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           __threadfence();
           __syncwarp();
           const size_t ci =
-              ((((size_t)it.j * d.n_qtiles + it.qt()) * p.n_heads + it.h) * kQTiles + a) * 4 + (warp & 3);
+              ((((size_t)it.j * d.n_qtiles + it.qt()) * p.n_heads + it.h) * kQTiles + a) * kFixPerTile + (warp & 3);
           int last = 0;
-          if (lane == 0) last = atomicAdd(p.fix_count + ci, 1) == pieces - 1;
+          if (lane == 0 && index_ok(ci < (size_t)p.fix_slots && part_ok, p.status))
+            last = atomicAdd(p.fix_count + ci, 1) == pieces - 1;
           last = __shfl_sync(0xffffffffu, last, 0);
           if (last) {
             if (lane == 0) p.fix_count[ci] = 0;
@@ -604,7 +633,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_before_sync();
   __syncthreads();
   cluster_sync_all();
-  if (warp == kMmaWarpP) {
+  if (warp == kPvWarp) {
     tc_fence_after_sync();
     tmem_dealloc_pair(tmem, 512);
   }

@@ -38,6 +38,12 @@ struct TileIter {
     run_row0 = r.row_begin[run];
     run_rows = r.rows[run];
   }
+  // debug builds: the current run lies inside the K/V planes, and so does head h's plane
+  __device__ __forceinline__ void check_run(const AttnParams& p) const {
+    index_ok(run_row0 >= 0 && run_rows > 0 && (int64_t)run_row0 + run_rows <= p.plane_rows && h >= 0 &&
+                 h < p.n_heads && p.plane_k + h < p.planes && p.plane_v + h < p.planes,
+             p.status);
+  }
   __device__ void init(const Decomp& d, const QueryUnits& u, const KeyRuns& r, const Range& rg) {
     g = 0;
     len = rg.len;
@@ -98,7 +104,7 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
   return false;
 }
 
-// Merge of the partials of one row of an item cut between CTAs:
+// Merge of the partials of one row of an item cut between workers:
 //   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
 // Piece k was written by CTA c_first + k of the lane: its last item for k = 0
 // (unless the item starts exactly at that CTA's range), its first item
@@ -106,11 +112,14 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint6
 // through L2 only.
 template <int D>
 static __device__ __noinline__ void merge_row(const AttnParams& p, int lane_i, int c_first, int pieces, int end0, int r,
-                                       uint16_t* dst) {
+                                              uint16_t* dst) {
   constexpr int kCached = 8;                 // pieces whose (m, l) stay in registers
   auto row_of = [&](int k) -> size_t {
     return partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0) * kItemRows + r;
   };
+  if (!index_ok(partial_slot(p.dec, lane_i, c_first + pieces - 1, 0) < (size_t)p.part_slots && r < kItemRows,
+                p.status))
+    return;
   // every piece's (reference max, sum): independent loads, one round trip
   float2 ml[kCached];
   float m_all = -INFINITY;

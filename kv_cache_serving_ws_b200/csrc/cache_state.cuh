@@ -87,6 +87,7 @@ struct ws_cache {
   EventPool ev_attn, ev_comb, ev_lat;
   int last_split = 0, last_ctas = 0;
   int64_t last_keys = 0;
+  int last_kernel = 0;
 };
 
 namespace ws {

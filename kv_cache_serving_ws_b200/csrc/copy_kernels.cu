@@ -34,6 +34,10 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 __global__ void __launch_bounds__(kCopyThreads) append_kernel(const __grid_constant__ AppendParams p) {
   const int l = blockIdx.y >> 1;
   const int kv = blockIdx.y & 1;
+  if (!index_ok(((int64_t)(p.layer0 + l) * 2 + kv + 1) * p.n_heads <= p.planes && p.row0 >= 0 &&
+                    p.row0 + p.n_tokens <= p.plane_rows,
+                p.status))
+    return;
   const int vpr = p.head_dim >> 3;          // 16-byte vectors per head row
   const int row_vecs = p.n_heads * vpr;     // vectors per token
   const uint4* src = reinterpret_cast<const uint4*>(kv ? p.src_v : p.src_k) + (size_t)l * p.n_tokens * row_vecs;
@@ -68,6 +72,10 @@ __global__ void __launch_bounds__(kCopyThreads) append_kernel(const __grid_const
 // blockIdx.y = kv; copies rows row0 .. row0+n-1 of one layer back to [n][H][D].
 __global__ void __launch_bounds__(kCopyThreads) read_kernel(const __grid_constant__ ReadParams p) {
   const int kv = blockIdx.y;
+  if (!index_ok(((int64_t)p.layer * 2 + kv + 1) * p.n_heads <= p.planes && p.row0 >= 0 &&
+                    p.row0 + p.n_tokens <= p.plane_rows,
+                p.status))
+    return;
   const int vpr = p.head_dim >> 3;
   const int row_vecs = p.n_heads * vpr;
   uint4* dst = reinterpret_cast<uint4*>(kv ? p.dst_v : p.dst_k);

@@ -81,6 +81,27 @@ __host__ __device__ inline size_t partial_slot(const Decomp& d, int lane, int ct
   return ((size_t)lane * d.lane_ctas + cta) * 2 + end;
 }
 
+// Device status values written by kernels into a status word (read by ws_sync).
+constexpr int kStatusTimeout = 1;   // a bounded wait ran out
+constexpr int kStatusIndex = 2;     // a device index check failed (WS_DEBUG_CHECKS builds)
+
+// Device index checks.  A build with -DWS_DEBUG_CHECKS (libws_debug.so) tests every
+// computed cache row, output row, partial slot and merge counter against the bounds
+// the host passes; a failed check records kStatusIndex in the status word and the
+// access is skipped (no trap, no fault).  In the normal build the checks compile away.
+#ifdef WS_DEBUG_CHECKS
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool index_ok(bool ok, int* status) {
+  if (kDebugChecks && !ok) {
+    if (status) atomicCAS(status, 0, kStatusIndex);
+    return false;
+  }
+  return true;
+}
+
 struct AttnParams {
   int32_t n_heads;          // H
   int32_t plane_k;          // KV-map plane index of head 0's K of this layer
@@ -94,6 +115,12 @@ struct AttnParams {
   int* status;              // device status word
   uint64_t timeout_ns;      // bound of every wait
   int32_t debug_skip_v_tile;  // test hook: never load V of this CTA-local tile (-1 = off)
+  // bounds for the index checks of debug builds
+  int64_t out_rows;         // rows of out (n_units * Nq)
+  int64_t part_slots;       // partial slots behind part_o / part_ml
+  int64_t fix_slots;        // merge counters behind fix_count
+  int64_t plane_rows;       // rows of each K/V plane
+  int64_t planes;           // planes of the K/V maps
   Decomp dec;
   QueryUnits qu;
   KeyRuns runs;
@@ -109,15 +136,16 @@ inline int encode_kv_map(CUtensorMap* map, const void* kv, int head_dim, int64_t
 }
 int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int n_query);
 
-// The attention launch: head_dim 128 runs on pairs of SMs (attention_pair.cu)
-// when the device can hold the pairs, otherwise -- and for head_dim 64 -- the
-// single-SM kernel (attention.cu).  `kv_map` has whole-tile boxes, `k_half_map`
-// boxes of 64 rows.  `p.dec` must come from decompose() with
-// attention_workers(head_dim) workers.
+// The attention launch: the single-SM kernel (attention.cu) for both head sizes,
+// or, with WS_ATTENTION_KERNEL=pair and head_dim 128, the kernel on pairs of SMs
+// (attention_pair.cu) where the device can hold its clusters.  `kv_map` has
+// whole-tile boxes, `k_half_map` boxes of 64 rows.  `p.dec` must come from
+// decompose() with attention_workers(head_dim) workers.
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const CUtensorMap& k_half_map,
                              const AttnParams& p, int head_dim, int* ctas, cudaStream_t stream);
 // Workers (CTAs, or CTA pairs) of the kernel launch_attention uses for head_dim.
 int attention_workers(int head_dim);
+bool attention_uses_pairs(int head_dim);
 // CTA pairs that can be resident at once for the paired kernel (0: none).
 int pair_workers();
 cudaError_t launch_attention_pair(const CUtensorMap& q_map, const CUtensorMap& k_map, const CUtensorMap& v_map,
@@ -136,9 +164,11 @@ cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream)
 // iterations (the separate merge launch then costs more).
 constexpr long long kFixupMinIterations = 64;
 inline bool use_fixup(const Decomp& d) { return lane_per(d, 0) >= kFixupMinIterations; }
-// Arrival counters of a call: one per (item, Q tile, warp of its softmax warpgroup).
+// Arrival counters of a call: kFixPerTile per (item, Q tile), one per softmax warp
+// that owns rows of the tile.
+constexpr int kFixPerTile = 4;
 inline int64_t fix_counters(int n_units, int n_qtiles, int heads) {
-  return (int64_t)n_units * n_qtiles * heads * kQTiles * 4;
+  return (int64_t)n_units * n_qtiles * heads * kQTiles * kFixPerTile;
 }
 
 // Copy a [L][n][H][D] token-major slice into the head-major cache planes:
@@ -154,6 +184,8 @@ struct AppendParams {
   int32_t head_dim;
   int64_t plane_rows;    // C*T
   int64_t row0;          // slot*T + segment offset
+  int64_t planes;        // planes of the cache (bound for debug builds)
+  int* status;           // device status word (debug builds' index checks)
 };
 cudaError_t launch_append(const AppendParams& p, cudaStream_t stream);
 
@@ -168,6 +200,8 @@ struct ReadParams {
   int32_t head_dim;
   int64_t plane_rows;
   int64_t row0;
+  int64_t planes;        // planes of the cache (bound for debug builds)
+  int* status;           // device status word (debug builds' index checks)
 };
 cudaError_t launch_read(const ReadParams& p, cudaStream_t stream);
 

@@ -166,6 +166,11 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)head_dim));
   p.out = out;
   p.timeout_ns = wait_bound_ns();
+  p.out_rows = n_query;
+  p.part_slots = (int64_t)slots;
+  p.fix_slots = (int64_t)(fix_bytes / sizeof(int));
+  p.plane_rows = n_keys;
+  p.planes = (int64_t)2 * n_heads;
   {
     std::lock_guard<std::mutex> lock(g_setup_mutex);
     p.debug_skip_v_tile = g_stall_tile;
@@ -218,9 +223,9 @@ extern "C" int ws_attention_noalloc_sync(cudaStream_t stream) {
     st = WS_ERR_CUDA;
   } else if (s != 0) {
     const int zero = 0;
-    st = cudaMemcpyToSymbol(g_scratch, &zero, sizeof(int), 0, cudaMemcpyHostToDevice) == cudaSuccess
-             ? WS_ERR_DEVICE_TIMEOUT
-             : WS_ERR_CUDA;
+    st = cudaMemcpyToSymbol(g_scratch, &zero, sizeof(int), 0, cudaMemcpyHostToDevice) != cudaSuccess
+             ? WS_ERR_CUDA
+             : (s == ws::kStatusIndex ? WS_ERR_DEVICE_CHECK : WS_ERR_DEVICE_TIMEOUT);
   }
   nvtxRangePop();
   return st;

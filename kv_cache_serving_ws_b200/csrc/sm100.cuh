@@ -5,6 +5,7 @@
 #include <cstdint>
 #include <cuda.h>
 
+#include "kernels.cuh"
 #include "tmem_ldst.cuh"
 
 namespace ws {
@@ -43,9 +44,6 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-
-// Device status values written by kernels into the library's status word.
-constexpr int kStatusTimeout = 1;
 
 // Every wait in the library's kernels is bounded.  `abort_flag` (shared memory)
 // is raised by the first thread whose wait runs out; the others see it and
@@ -196,6 +194,12 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 // releasing this thread's prior writes at cluster scope.
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+// Arrive with no memory ordering: for barriers whose data is ordered otherwise
+// (TMEM through tcgen05.wait and the tcgen05 thread-sync fences, copies through
+// their transaction bytes), where the arrival is only a count.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // Phase test that acquires at cluster scope (the barrier's arrivals may come from the peer CTA).
 __device__ __forceinline__ uint32_t mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {

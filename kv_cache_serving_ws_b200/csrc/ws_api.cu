@@ -234,6 +234,8 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
     a.head_dim = D;
     a.plane_rows = h->session_rows * h->n_sessions;
     a.row0 = sessions[j] * h->session_rows + (int64_t)slot * h->T + h->cfg.n_cond;
+    a.planes = (int64_t)L * 2 * H;
+    a.status = h->d_status;
     cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_lat.next() : nullptr;
     if (ev) cudaEventRecord(ev[0], stream);
     if (launch_append(a, stream) != cudaSuccess) return WS_ERR_CUDA;
@@ -253,6 +255,11 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   p.fix_count = h->d_fix;
   p.timeout_ns = h->timeout_ns;
   p.debug_skip_v_tile = h->debug_skip_v_tile;
+  p.out_rows = (int64_t)n * h->Nq;
+  p.part_slots = h->slot_cap;
+  p.fix_slots = (int64_t)(h->fix_bytes / sizeof(int));
+  p.plane_rows = h->session_rows * h->n_sessions;
+  p.planes = (int64_t)L * 2 * H;
   cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_attn.next() : nullptr;
   if (ev) cudaEventRecord(ev[0], stream);
   int ctas = 0;
@@ -267,6 +274,7 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   h->last_split = p.dec.lane_ctas;
   h->last_ctas = ctas;
   h->last_keys = keys;
+  h->last_kernel = attention_uses_pairs(D) ? 2 : 1;
   return WS_OK;
 }
 
@@ -298,6 +306,8 @@ int append_impl(ws_cache* h, int session, int64_t unit, int seg, const uint16_t*
   p.head_dim = h->cfg.head_dim;
   p.plane_rows = h->session_rows * h->n_sessions;
   p.row0 = session * h->session_rows + (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  p.planes = (int64_t)h->cfg.n_layers * 2 * h->cfg.n_heads;
+  p.status = h->d_status;
   const cudaError_t e = launch_append(p, stream);
   if (e != cudaSuccess) return WS_ERR_CUDA;
   if (seg == WS_SEG_COND) {
@@ -338,6 +348,7 @@ const char* ws_status_string(int status) {
     case WS_ERR_CUDA: return "CUDA error";
     case WS_ERR_DEVICE_TIMEOUT: return "a kernel's bounded wait ran out";
     case WS_ERR_UNSUPPORTED: return "request outside what this build supports";
+    case WS_ERR_DEVICE_CHECK: return "a device-side index check failed (debug build)";
     default: return "unknown status";
   }
 }
@@ -493,6 +504,8 @@ int ws_session_read(ws_cache_t* h, int32_t session, int layer, int64_t unit, int
   p.head_dim = h->cfg.head_dim;
   p.plane_rows = h->session_rows * h->n_sessions;
   p.row0 = session * h->session_rows + (int64_t)slot * h->T + (seg == WS_SEG_COND ? 0 : h->cfg.n_cond);
+  p.planes = (int64_t)h->cfg.n_layers * 2 * h->cfg.n_heads;
+  p.status = h->d_status;
   return cuda_status(launch_read(p, stream));
 }
 
@@ -559,7 +572,7 @@ int ws_sync(ws_cache_t* h, cudaStream_t stream) {
     // a kernel that gave up may have left merge counters mid-count
     if (cudaMemset(h->d_status, 0, sizeof(int)) != cudaSuccess) return WS_ERR_CUDA;
     if (cudaMemset(h->d_fix, 0, h->fix_bytes) != cudaSuccess) return WS_ERR_CUDA;
-    return WS_ERR_DEVICE_TIMEOUT;
+    return s == kStatusIndex ? WS_ERR_DEVICE_CHECK : WS_ERR_DEVICE_TIMEOUT;
   }
   return WS_OK;
 }
@@ -600,6 +613,7 @@ int ws_profile_read(ws_cache_t* h, ws_profile* out) {
   out->last_n_split = h->last_split;
   out->last_ctas = h->last_ctas;
   out->last_keys = h->last_keys;
+  out->last_kernel = h->last_kernel;
   return WS_OK;
 }
 

@@ -16,7 +16,8 @@ import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-LIB_PATH = os.path.join(HERE, "libws.so")
+# WS_LIBRARY=debug loads the build with device index checks (libws_debug.so).
+LIB_PATH = os.path.join(HERE, "libws_debug.so" if os.environ.get("WS_LIBRARY") == "debug" else "libws.so")
 SYNTH_PATH = os.path.join(HERE, "libws_synth.so")
 HEADER = os.path.join(ROOT, "include", "ws.h")
 
@@ -30,6 +31,7 @@ WS_ERR_NOT_READY = -6
 WS_ERR_CUDA = -7
 WS_ERR_DEVICE_TIMEOUT = -8
 WS_ERR_UNSUPPORTED = -9
+WS_ERR_DEVICE_CHECK = -10
 WS_SEG_COND = 0
 WS_SEG_LATENT = 1
 
@@ -50,7 +52,8 @@ class ws_profile(C.Structure):
     _fields_ = [("attention_launches", C.c_int64), ("attention_ms", C.c_double),
                 ("combine_launches", C.c_int64), ("combine_ms", C.c_double),
                 ("latent_write_launches", C.c_int64), ("latent_write_ms", C.c_double),
-                ("last_n_split", C.c_int32), ("last_ctas", C.c_int32), ("last_keys", C.c_int64)]
+                ("last_n_split", C.c_int32), ("last_ctas", C.c_int32), ("last_keys", C.c_int64),
+                ("last_kernel", C.c_int32)]
 
 
 class ws_unit_io(C.Structure):
@@ -120,7 +123,8 @@ def lib():
     global _lib
     if _lib is None:
         if not os.path.exists(LIB_PATH):
-            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_serving_ws_b200.build`")
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_serving_ws_b200.build`"
+                               + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
         _lib = C.CDLL(LIB_PATH)
         _declare(_lib)
     return _lib
