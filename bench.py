@@ -33,9 +33,10 @@ METRIC = "block-causal unit-attention TFLOP/s & ms per 640×368 unit on 1 B200 (
 UNIT = "TFLOP/s"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "unit_attention_traffic.txt")
-KERNEL_SOURCES = ["kv_cache_serving_ws_b200/csrc/attention.cu", "kv_cache_serving_ws_b200/csrc/attention_pair.cu",
-                  "kv_cache_serving_ws_b200/csrc/attn_common.cuh", "kv_cache_serving_ws_b200/csrc/sm100.cuh",
-                  "kv_cache_serving_ws_b200/csrc/kernels.cuh", "kv_cache_serving_ws_b200/csrc/tmem_ldst.cuh"]
+# sources of the benchmark's attention kernel (the single-SM kernel)
+KERNEL_SOURCES = ["kv_cache_serving_ws_b200/csrc/attention.cu", "kv_cache_serving_ws_b200/csrc/attn_common.cuh",
+                  "kv_cache_serving_ws_b200/csrc/sm100.cuh", "kv_cache_serving_ws_b200/csrc/kernels.cuh",
+                  "kv_cache_serving_ws_b200/csrc/tmem_ldst.cuh"]
 
 
 # ------------------------------------------------------------ multi-rank --
