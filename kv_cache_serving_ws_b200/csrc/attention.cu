@@ -38,6 +38,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <string>
+#include <type_traits>
 
 #include "attn_common.cuh"
 #include "kernels.cuh"
@@ -503,53 +504,85 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Merge of the partials of items cut between CTAs as a separate launch (calls
 // whose CTAs run few iterations, see AttnParams::fixup):
 //   out = sum_k 2^(m_k - M) O_k / sum_k 2^(m_k - M) l_k,   M = max_k m_k.
-// One warp per (row, head); each lane owns D/32 consecutive columns.
+// One warp per output row, each lane D/32 consecutive columns; a block takes 8 rows
+// of one item (query unit j, query block qt, head h).  The kernel is latency-bound
+// (one or two waves of short warps), so a warp issues its loads in one round trip:
+// lane k loads piece k's (max, sum) pair while every lane loads its columns of the
+// first kPre pieces' partial rows; the weights then come from warp shuffles.
+constexpr int kMergeRowsPerBlock = 8;
 template <int D>
-__global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(32 * kMergeRowsPerBlock) merge_kernel(const __grid_constant__ AttnParams p) {
   constexpr int kPer = D / 32;
-  const int gw = (int)((blockIdx.x * (size_t)blockDim.x + threadIdx.x) >> 5);
+  constexpr int kPre = 4;
+  constexpr int kChunks = kItemRows / kMergeRowsPerBlock;
+  using Vec = typename std::conditional<kPer == 4, float4, float2>::type;
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int rows = p.qu.n_units * p.qu.rows;
-  if (gw >= rows * p.n_heads) return;
-  const int row = gw / p.n_heads;
-  const int h = gw - row * p.n_heads;
-  const int j = row / p.qu.rows;
-  const int r_unit = row - j * p.qu.rows;
-  const int qt = r_unit / kItemRows;
-  const int r = r_unit - qt * kItemRows;
+  const int item = blockIdx.x / kChunks;                   // (j * n_qtiles + qt) * H + h
+  const int chunk = blockIdx.x - item * kChunks;
+  const int h = item % p.n_heads;
+  const int jq = item / p.n_heads;
+  const int qt = jq % p.dec.n_qtiles;
+  const int j = jq / p.dec.n_qtiles;
   int lane_i, c_first, pieces, end0;
   item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
-  if (pieces == 1) return;                       // written directly by its CTA
-  if (!index_ok(partial_slot(p.dec, lane_i, c_first + pieces - 1, 0) < (size_t)p.part_slots &&
-                    (int64_t)row < p.out_rows,
+  if (pieces == 1) return;                                 // written directly by its CTA
+  const int r = chunk * kMergeRowsPerBlock + warp;         // row within the item's block
+  const int r_unit = qt * kItemRows + r;
+  if (r_unit >= p.qu.rows) return;
+  const int64_t row = (int64_t)j * p.qu.rows + r_unit;
+  if (!index_ok(partial_slot(p.dec, lane_i, c_first + pieces - 1, 0) < (size_t)p.part_slots && row < p.out_rows,
                 p.status))
     return;
-  // piece k was written by CTA c_first + k: its last item for k = 0 (unless
-  // the item starts exactly at that CTA's range), its first item otherwise
-  float m_all = -INFINITY;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    m_all = fmaxf(m_all, p.part_ml[(slot * kItemRows + r) * 2]);
-  }
-  float l_all = 0.f;
+  // piece k was written by CTA c_first + k: its last item for k = 0 (unless the
+  // item starts exactly at that CTA's range), its first item otherwise
+  auto prow_of = [&](int k) -> size_t {
+    return partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0) * kItemRows + r;
+  };
+  auto load_cols = [&](int k) -> Vec {
+    return __ldcg(reinterpret_cast<const Vec*>(p.part_o + prow_of(k) * D) + lane);
+  };
+  auto fma_cols = [](float* acc, float w, const Vec& v) {
+    if constexpr (kPer == 4) {
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+      acc[0] += w * v.x; acc[1] += w * v.y;
+    }
+  };
+  // 1. one round trip: (m, l) of pieces 0..31 and the first kPre partial rows
+  const float2 ml0 = lane < pieces ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + prow_of(lane) * 2))
+                                   : make_float2(-INFINITY, 0.f);
+  Vec pre[kPre];
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) pre[k] = k < pieces ? load_cols(k) : Vec{};
+  // 2. M over all pieces (more than 32 only for very small per-CTA ranges)
+  float m_all = ml0.x;
+  for (int k0 = 32; k0 < pieces; k0 += 32)
+    if (k0 + lane < pieces) m_all = fmaxf(m_all, __ldcg(p.part_ml + prow_of(k0 + lane) * 2));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m_all = fmaxf(m_all, __shfl_xor_sync(0xffffffffu, m_all, o));
+  // 3. weights 2^(m_k - M), the weighted rows and the weighted sums
+  float w = lane < pieces ? ex2_approx(ml0.x - m_all) : 0.f;
+  float l_all = w * ml0.y;
   float acc[kPer];
 #pragma unroll
   for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  for (int k = 0; k < pieces; ++k) {
-    const size_t slot = partial_slot(p.dec, lane_i, c_first + k, k == 0 ? end0 : 0);
-    const size_t prow = slot * kItemRows + r;
-    const float2 ml = *reinterpret_cast<const float2*>(p.part_ml + prow * 2);
-    const float w = ex2_approx(ml.x - m_all);
+#pragma unroll
+  for (int k = 0; k < kPre; ++k) fma_cols(acc, __shfl_sync(0xffffffffu, w, k), pre[k]);
+  const int n0 = pieces < 32 ? pieces : 32;
+#pragma unroll 4
+  for (int k = kPre; k < n0; ++k) fma_cols(acc, __shfl_sync(0xffffffffu, w, k), load_cols(k));
+  for (int k0 = 32; k0 < pieces; k0 += 32) {
+    const int n = pieces - k0 < 32 ? pieces - k0 : 32;
+    const float2 ml = lane < n ? __ldcg(reinterpret_cast<const float2*>(p.part_ml + prow_of(k0 + lane) * 2))
+                               : make_float2(-INFINITY, 0.f);
+    w = lane < n ? ex2_approx(ml.x - m_all) : 0.f;
     l_all += w * ml.y;
-    const float* po = p.part_o + prow * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      const float4 o = *reinterpret_cast<const float4*>(po);
-      acc[0] += w * o.x; acc[1] += w * o.y; acc[2] += w * o.z; acc[3] += w * o.w;
-    } else {
-      const float2 o = *reinterpret_cast<const float2*>(po);
-      acc[0] += w * o.x; acc[1] += w * o.y;
-    }
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) fma_cols(acc, __shfl_sync(0xffffffffu, w, k), load_cols(k0 + k));
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l_all += __shfl_xor_sync(0xffffffffu, l_all, o);
   const float inv = 1.f / l_all;
   uint16_t* dst = p.out + ((size_t)row * p.n_heads + h) * D + lane * kPer;
   if constexpr (kPer == 4) {
@@ -656,12 +689,12 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
 }
 
 cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
-  const long long warps = (long long)p.qu.n_units * p.qu.rows * p.n_heads;
-  const int grid = (int)((warps * 32 + 255) / 256);
+  const long long items = (long long)p.qu.n_units * p.dec.n_qtiles * p.n_heads;
+  const int grid = (int)(items * (kItemRows / kMergeRowsPerBlock));
   if (head_dim == 128)
-    merge_kernel<128><<<grid, 256, 0, stream>>>(p);
+    merge_kernel<128><<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(p);
   else if (head_dim == 64)
-    merge_kernel<64><<<grid, 256, 0, stream>>>(p);
+    merge_kernel<64><<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(p);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();

@@ -61,8 +61,14 @@ __host__ __device__ inline int lane_qtiles(const Decomp& d, int lane) {
 __host__ __device__ inline long long lane_work(const Decomp& d, int lane) {
   return (long long)lane_qtiles(d, lane) * d.heads * d.tiles;
 }
+// Quotient of non-negative a by positive b; 32-bit division when both fit (the
+// common case: a 64-bit division is a long instruction sequence on the GPU).
+__host__ __device__ inline long long div_nonneg(long long a, long long b) {
+  if (a >= 0 && a <= 0x7fffffffLL && b <= 0x7fffffffLL) return (long long)((unsigned)a / (unsigned)b);
+  return a / b;
+}
 __host__ __device__ inline long long lane_per(const Decomp& d, int lane) {
-  return (lane_work(d, lane) + d.lane_ctas - 1) / d.lane_ctas;
+  return div_nonneg(lane_work(d, lane) + d.lane_ctas - 1, d.lane_ctas);
 }
 // The CTAs (lane-local) that cover item (j, qt, h), and the partial slot index
 // of its first piece (0 when the item starts exactly at that CTA's range).
@@ -73,8 +79,8 @@ __host__ __device__ inline void item_span(const Decomp& d, const QueryUnits& u, 
   const long long start = ((long long)h * lane_qtiles(d, lane) + a) * d.tiles + u.tile_start[j];
   const int len = u.tile_start[j + 1] - u.tile_start[j];
   const long long per = lane_per(d, lane);
-  first_cta = (int)(start / per);
-  pieces = (int)((start + len - 1) / per) - first_cta + 1;
+  first_cta = (int)div_nonneg(start, per);
+  pieces = (int)(len > 0 ? div_nonneg(start + len - 1, per) : (start + len - 1) / per) - first_cta + 1;
   first_slot_end = start == (long long)first_cta * per ? 0 : 1;
 }
 __host__ __device__ inline size_t partial_slot(const Decomp& d, int lane, int cta, int end) {
