@@ -107,7 +107,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long end = rg.start + per < work ? rg.start + per : work;
     rg.len = end > rg.start ? (int)(end - rg.start) : 0;
   }
-  if (rg.len == 0) return;                 // whole CTA: nothing allocated yet
+  if (rg.len == 0) {                       // whole CTA: nothing allocated yet
+    griddep_wait();                        // (every CTA completes after the previous grid)
+    return;
+  }
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
@@ -155,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const WaitGuard guard{abort_flag, p.status, p.timeout_ns};
+  griddep_wait();   // Q, the cache and the partials may be in use by the previous kernel
 
   if (warp >= kSoftmaxWarps) {
     if (warp == kProducerWarp && lane == 0) {
@@ -493,6 +497,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  griddep_launch_dependents();
   tc_fence_before_sync();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -520,16 +525,17 @@ __global__ void __launch_bounds__(32 * kMergeRowsPerBlock) merge_kernel(const __
   const int lane = threadIdx.x & 31;
   const int item = blockIdx.x / kChunks;                   // (j * n_qtiles + qt) * H + h
   const int chunk = blockIdx.x - item * kChunks;
+  griddep_launch_dependents();
   const int h = item % p.n_heads;
   const int jq = item / p.n_heads;
   const int qt = jq % p.dec.n_qtiles;
   const int j = jq / p.dec.n_qtiles;
   int lane_i, c_first, pieces, end0;
   item_span(p.dec, p.qu, j, qt, h, lane_i, c_first, pieces, end0);
-  if (pieces == 1) return;                                 // written directly by its CTA
   const int r = chunk * kMergeRowsPerBlock + warp;         // row within the item's block
   const int r_unit = qt * kItemRows + r;
-  if (r_unit >= p.qu.rows) return;
+  griddep_wait();                                          // the partials of the attention kernel
+  if (pieces == 1 || r_unit >= p.qu.rows) return;          // pieces == 1: written directly by its CTA
   const int64_t row = (int64_t)j * p.qu.rows + r_unit;
   if (!index_ok(partial_slot(p.dec, lane_i, c_first + pieces - 1, 0) < (size_t)p.part_slots && row < p.out_rows,
                 p.status))
@@ -652,8 +658,8 @@ static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMa
   }
   const int grid = p.dec.lanes * p.dec.lane_ctas;
   if (ctas) *ctas = grid;
-  unit_attention_kernel<D><<<grid, kThreads, Smem<D>::kAlloc, stream>>>(q_map, kv_map, p);
-  const cudaError_t e = cudaGetLastError();
+  PdlLaunch l(dim3(grid), dim3(kThreads), Smem<D>::kAlloc, stream);
+  const cudaError_t e = cudaLaunchKernelEx(&l.cfg, unit_attention_kernel<D>, q_map, kv_map, p);
   if (e != cudaSuccess && std::getenv("WS_DEBUG")) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, unit_attention_kernel<D>);
@@ -691,13 +697,10 @@ cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map
 cudaError_t launch_merge(const AttnParams& p, int head_dim, cudaStream_t stream) {
   const long long items = (long long)p.qu.n_units * p.dec.n_qtiles * p.n_heads;
   const int grid = (int)(items * (kItemRows / kMergeRowsPerBlock));
-  if (head_dim == 128)
-    merge_kernel<128><<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(p);
-  else if (head_dim == 64)
-    merge_kernel<64><<<grid, 32 * kMergeRowsPerBlock, 0, stream>>>(p);
-  else
-    return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  PdlLaunch l(dim3(grid), dim3(32 * kMergeRowsPerBlock), 0, stream);
+  if (head_dim == 128) return cudaLaunchKernelEx(&l.cfg, merge_kernel<128>, p);
+  if (head_dim == 64) return cudaLaunchKernelEx(&l.cfg, merge_kernel<64>, p);
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace ws

@@ -32,6 +32,8 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 
 // blockIdx.y = l*2 + kv (layer of the slice, K or V); blockIdx.x strides over tokens.
 __global__ void __launch_bounds__(kCopyThreads) append_kernel(const __grid_constant__ AppendParams p) {
+  griddep_wait();                 // the slice may come from the previous kernel of the stream
+  griddep_launch_dependents();
   const int l = blockIdx.y >> 1;
   const int kv = blockIdx.y & 1;
   if (!index_ok(((int64_t)(p.layer0 + l) * 2 + kv + 1) * p.n_heads <= p.planes && p.row0 >= 0 &&
@@ -119,8 +121,8 @@ cudaError_t launch_append(const AppendParams& p, cudaStream_t stream) {
   if (gx * pairs > want) gx = (want + pairs - 1) / pairs;
   if (gx < 1) gx = 1;
   dim3 grid(gx, pairs);
-  append_kernel<<<grid, kCopyThreads, 0, stream>>>(p);
-  return cudaGetLastError();
+  PdlLaunch l(grid, dim3(kCopyThreads), 0, stream);
+  return cudaLaunchKernelEx(&l.cfg, append_kernel, p);
 }
 
 cudaError_t launch_read(const ReadParams& p, cudaStream_t stream) {

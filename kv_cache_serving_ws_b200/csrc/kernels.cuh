@@ -213,6 +213,35 @@ cudaError_t launch_read(const ReadParams& p, cudaStream_t stream);
 
 cudaError_t launch_euler(uint16_t* x, const uint16_t* v, float dt, int64_t n, cudaStream_t stream);
 
+// Programmatic dependent launch.  The append, attention and merge kernels of a call
+// are launched with programmatic stream serialization: a kernel may start while the
+// previous kernel of the stream is finishing, runs its prologue (barrier setup,
+// tensor-memory allocation, index arithmetic on its parameters: no global memory),
+// then waits in griddep_wait() until the previous grid has completed and its writes
+// are visible.  Every thread that touches global memory passes that wait.  A kernel
+// calls griddep_launch_dependents() once its own prologue or main loop is done, so
+// the next kernel's launch overlaps its tail; the next kernel can only start once
+// every CTA of this one has been scheduled (so it cannot take an SM that one of them
+// still needs).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg{};
+  cudaLaunchAttribute attr[1];
+  PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t stream) {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+
 // Host helpers.  Kernel attributes and SM counts are per device: a process may
 // drive several GPUs, so every cached value is kept per device ordinal.
 constexpr int kMaxDevices = 64;
