@@ -259,8 +259,9 @@ def run_ours(args, rank, local_rank, world):
     roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": pk["bf16_sustained"], "unit": "TFLOP/s",
                 "frac": round(achieved / pk["bf16_sustained"], 4), "traffic": traffic,
                 "peak_kind": f"{pk['source']} bf16 dense, sustained (kernel timed inside a long step)"}
-    # conditioning, commit; latent write + attention per call; Euler; separate merges if any
-    launches_per_step = 2 + L * S * 2 + S + prof["combine_launches"] // max(1, args.steps)
+    # conditioning, commit; per call the attention, a latent write when the kernel does
+    # not fold it in, a merge when items were cut; Euler
+    launches_per_step = 2 + S + (n_attn + prof["latent_write_launches"] + prof["combine_launches"]) // max(1, args.steps)
 
     # ---- HBM-bound kernels, timed on their own on the same stream
     extra = hbm_kernels(ws, g, w, torch, dev, pk, x, vel, commit_k, commit_v, cond_k, cond_v, next_unit)
@@ -618,7 +619,7 @@ def percentiles(xs):
 def run_schedule(args):
     """Per-unit schedule of the whole unit (conditioning append, 40 layers x 4 Euler
     steps of attention, commit), units back to back and paced at the stream's 160 ms
-    cadence.  Direct calls (~490 launches per unit) against the unit program (one CUDA
+    cadence.  Direct calls (one launch per layer call plus a few per unit) against the unit program (one CUDA
     graph per unit, updated in place).  Reports per-unit device time percentiles, the
     host time the program spends recording a unit, and, paced, the latency from a
     unit's release (its conditioning slice copied from pinned host memory) to its
@@ -735,7 +736,7 @@ def run_schedule(args):
             "mode": "schedule", "workload": w.name, "units": n, "unit_budget_ms": period_s * 1e3,
             "tflop_per_unit": round(flops_unit / 1e12, 2),
             "direct": {"unit_ms": percentiles(per_direct), "host_ms_per_unit": round(host_direct, 3),
-                       "launches_per_unit": 2 + L * S * 2 + S},
+                       "launches_per_unit": 2 + S + L * S * (1 if ws.ws_profile_read(g.h)["last_kernel"] == 1 else 2)},
             "graph": {"unit_ms": percentiles(per_graph), "host_ms_per_unit": round(host_graph, 3),
                       "record_ms_per_unit": round((s1["record_ms"] - s0["record_ms"]) / max(1, n + 3), 3),
                       "kernel_nodes": s1["nodes"], "updates_in_place": upd, "instantiations": inst,

@@ -66,9 +66,10 @@ enum Bar : int {
 constexpr int kSoftmaxWarps = 4 * kQTiles;
 constexpr int kProducerWarp = kSoftmaxWarps;
 constexpr int kMmaWarp = kSoftmaxWarps + 1;
-// 320 threads, one CTA per SM: three warps share some SM sub-partitions, which
+constexpr int kCopyWarp = kSoftmaxWarps + 2;   // writes the call's latent K/V into the cache
+// 352 threads, one CTA per SM: three warps share some SM sub-partitions, which
 // caps a thread at 168 registers; the softmax fits without spills.
-constexpr int kThreads = 32 * (kSoftmaxWarps + 2);
+constexpr int kThreads = 32 * (kSoftmaxWarps + 3);
 constexpr int kTmemCols = 512;
 constexpr int kRowBytes = 128;   // one 128-byte swizzle row = 64 bf16
 
@@ -90,9 +91,66 @@ struct Smem {
 __device__ __forceinline__ uint32_t tmem_s(uint32_t base, int a) { return base + (uint32_t)(a * 256); }
 __device__ __forceinline__ uint32_t tmem_o(uint32_t base, int a) { return base + (uint32_t)(a * 256 + 128); }
 
+// The latent write folded into the attention launch: the call's k_new / v_new token
+// rows [n_units*Nq][H][D] go to plane rows latent_row0[j] + t of planes plane_k + h
+// (K) and plane_v + h (V) -- the in-place cache write of the unit's K/V slice
+// ("Wan-Streamer v0.2：更高分辨率，相同延迟", paper.rainbus.top, section 前置知识, entry
+// K/V缓存预分片).  The key tiles of those rows are loaded from k_new / v_new anyway;
+// every whole tile is stored from shared memory by TMA (store_latent_tiles below), once
+// per (head, tile).  This function copies the rest: each unit's last Nq % 128 rows,
+// which no whole tile covers.  CTA b of the grid takes an equal share of those rows
+// (K rows, then V rows); `nthr` threads of it walk the share's 16-byte vectors, four
+// loads in flight per thread.  Nothing in the launch reads these cache rows.
+template <int D>
+__device__ void copy_latent_tail(const AttnParams& p, int tid, int nthr) {
+  constexpr int kVd = D / 8;                  // 16-byte vectors per head row
+  constexpr int kDepth = 4;
+  const int nq = p.qu.rows;
+  const int t0 = (nq / kBlockN) * kBlockN;    // first row not covered by a whole tile
+  const int tail = nq - t0;
+  const int rows_all = p.qu.n_units * tail;
+  const int row_vecs = p.n_heads * kVd;
+  const int total = 2 * rows_all;
+  if (total == 0) return;
+  const int per = (total + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int r0 = (int)blockIdx.x * per;
+  const int r1 = min(total, r0 + per);
+  if (r0 >= r1) return;
+  const int nv = (r1 - r0) * row_vecs;
+  for (int f0 = tid; f0 < nv; f0 += kDepth * nthr) {
+    uint4 v[kDepth];
+    uint4* dst[kDepth];
+#pragma unroll
+    for (int u = 0; u < kDepth; ++u) {
+      const int f = f0 + u * nthr;
+      dst[u] = nullptr;
+      if (f < nv) {
+        const int r = r0 + f / row_vecs;
+        const int e = f - (r - r0) * row_vecs;
+        const int kv = r >= rows_all ? 1 : 0;
+        const int rr = r - kv * rows_all;
+        const int j = rr / tail;
+        const int t = t0 + (rr - j * tail);   // row within unit j
+        const int64_t row = p.latent_row0[j] + t;
+        const int h = e / kVd;
+        const int64_t plane = (int64_t)(kv ? p.plane_v : p.plane_k) + h;
+        if (index_ok(row >= 0 && row < p.plane_rows && plane < p.planes, p.status)) {
+          const size_t tok = (size_t)j * nq + t;
+          v[u] = ld_global_nc_v4(reinterpret_cast<const uint4*>(kv ? p.v_new : p.k_new) + tok * row_vecs + e);
+          dst[u] = reinterpret_cast<uint4*>(p.cache + ((size_t)plane * p.plane_rows + row) * D) + (e - h * kVd);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kDepth; ++u)
+      if (dst[u]) *dst[u] = v[u];
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     unit_attention_kernel(const __grid_constant__ CUtensorMap q_map, const __grid_constant__ CUtensorMap kv_map,
+                          const __grid_constant__ CUtensorMap knew_map, const __grid_constant__ CUtensorMap vnew_map,
                           const __grid_constant__ AttnParams p) {
   using S = Smem<D>;
   const Decomp& d = p.dec;
@@ -109,6 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (rg.len == 0) {                       // whole CTA: nothing allocated yet
     griddep_wait();                        // (every CTA completes after the previous grid)
+    if (p.fold) copy_latent_tail<D>(p, threadIdx.x, kThreads);
     return;
   }
 
@@ -129,11 +188,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars[kQFull], 1);
     mbar_init(&bars[kQEmpty], 1);
+    // with the fold, a stage is free once the MMAs and the latent store are done with it
+    const uint32_t empty_count = p.fold ? 2 : 1;
     for (int s = 0; s < 2; ++s) {
       mbar_init(&bars[kKFull + s], 1);
-      mbar_init(&bars[kKEmpty + s], 1);
+      mbar_init(&bars[kKEmpty + s], empty_count);
       mbar_init(&bars[kVFull + s], 1);
-      mbar_init(&bars[kVEmpty + s], 1);
+      mbar_init(&bars[kVEmpty + s], empty_count);
     }
     for (int a = 0; a < kQTiles; ++a) {
       mbar_init(&bars[kSFull + a], 1);
@@ -152,6 +213,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kProducerWarp && lane == 0) {
     prefetch_tensormap(&q_map);
     prefetch_tensormap(&kv_map);
+    if (p.fold) {
+      prefetch_tensormap(&knew_map);
+      prefetch_tensormap(&vnew_map);
+    }
   }
   tc_fence_before_sync();
   __syncthreads();
@@ -183,16 +248,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         it.check_run(p);
         if (use > 0 && !wait_phase(&bars[kKEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
         mbar_arrive_expect_tx(&bars[kKFull + s], S::kTileBytes);
-        for (int c = 0; c < S::kChunks; ++c)
-          tma_load_3d(sK + s * S::kTileBytes + c * kBlockN * kRowBytes, &kv_map, &bars[kKFull + s], c * 64, row0,
-                      p.plane_k + it.h);
+        for (int c = 0; c < S::kChunks; ++c) {
+          uint8_t* dst = sK + s * S::kTileBytes + c * kBlockN * kRowBytes;
+          if (it.run_new)   // the call's own latent rows: k_new [rows][H][D]
+            tma_load_3d(dst, &knew_map, &bars[kKFull + s], c * 64, it.h, row0);
+          else
+            tma_load_3d(dst, &kv_map, &bars[kKFull + s], c * 64, row0, p.plane_k + it.h);
+        }
         last_k[s] = g;
         if (use > 0 && !wait_phase(&bars[kVEmpty + s], (use - 1) & 1, guard)) { ok = false; break; }
         if (g != p.debug_skip_v_tile) {
           mbar_arrive_expect_tx(&bars[kVFull + s], S::kTileBytes);
-          for (int c = 0; c < S::kChunks; ++c)
-            tma_load_3d(sV + s * S::kTileBytes + c * kBlockN * kRowBytes, &kv_map, &bars[kVFull + s], c * 64,
-                        row0, p.plane_v + it.h);
+          for (int c = 0; c < S::kChunks; ++c) {
+            uint8_t* dst = sV + s * S::kTileBytes + c * kBlockN * kRowBytes;
+            if (it.run_new)
+              tma_load_3d(dst, &vnew_map, &bars[kVFull + s], c * 64, it.h, row0);
+            else
+              tma_load_3d(dst, &kv_map, &bars[kVFull + s], c * 64, row0, p.plane_v + it.h);
+          }
           last_v[s] = g;
         }
       }
@@ -203,6 +276,43 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (last_k[s] >= 0) drain_wait(&bars[kKFull + s], ((uint32_t)last_k[s] >> 1) & 1, p.timeout_ns);
           if (last_v[s] >= 0) drain_wait(&bars[kVFull + s], ((uint32_t)last_v[s] >> 1) & 1, p.timeout_ns);
         }
+      }
+    } else if (warp == kCopyWarp && p.fold) {
+      // ------------------------------------------------- latent write (fold)
+      copy_latent_tail<D>(p, lane, 32);
+      __syncwarp();
+      if (lane == 0) {
+        // Follows the producer's stages: once a stage's K and V have landed, a whole
+        // tile of the call's own latent rows, seen by query block 0, is stored to its
+        // cache rows (each (head, tile) once); then the stage is released.
+        bool ok = true;
+        TileIter it;
+        it.init(d, p.qu, p.runs, rg);
+        for (int g = 0; g < len && ok; ++g, it.next(p.qu, p.runs)) {
+          const int s = g & 1;
+          const uint32_t ph = ((uint32_t)g >> 1) & 1;
+          const bool store = it.run_new && it.qt() == 0 && it.valid() == kBlockN;
+          const int64_t row = p.latent_row0[it.j] + (it.row0() - it.j * p.qu.rows);
+          const bool row_ok = !store || index_ok(row >= 0 && row + kBlockN <= p.plane_rows, p.status);
+          if (!wait_phase(&bars[kKFull + s], ph, guard)) { ok = false; break; }
+          if (store && row_ok) {
+            fence_proxy_async_smem();
+            for (int c = 0; c < S::kChunks; ++c)
+              tma_store_3d(&kv_map, sK + s * S::kTileBytes + c * kBlockN * kRowBytes, c * 64, (int32_t)row,
+                           p.plane_k + it.h);
+          }
+          if (!wait_phase(&bars[kVFull + s], ph, guard)) { ok = false; break; }
+          if (store && row_ok) {
+            for (int c = 0; c < S::kChunks; ++c)
+              tma_store_3d(&kv_map, sV + s * S::kTileBytes + c * kBlockN * kRowBytes, c * 64, (int32_t)row,
+                           p.plane_v + it.h);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
+          mbar_arrive(&bars[kKEmpty + s]);
+          mbar_arrive(&bars[kVEmpty + s]);
+        }
+        bulk_wait_group0();
       }
     } else if (warp == kMmaWarp) {
       // -------------------------------------------------------- MMA issuer
@@ -644,8 +754,9 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 }
 
 template <int D>
-static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMap& kv_map, const AttnParams& p,
-                                      int* ctas, cudaStream_t stream) {
+static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMap& kv_map,
+                                      const CUtensorMap* new_maps, const AttnParams& p, int* ctas,
+                                      cudaStream_t stream) {
   // the shared-memory opt-in is a per-device attribute of the kernel
   static std::atomic<bool> configured[kMaxDevices];
   const int dev = current_device();
@@ -659,7 +770,10 @@ static cudaError_t launch_attention_d(const CUtensorMap& q_map, const CUtensorMa
   const int grid = p.dec.lanes * p.dec.lane_ctas;
   if (ctas) *ctas = grid;
   PdlLaunch l(dim3(grid), dim3(kThreads), Smem<D>::kAlloc, stream);
-  const cudaError_t e = cudaLaunchKernelEx(&l.cfg, unit_attention_kernel<D>, q_map, kv_map, p);
+  // without the fold the k_new / v_new maps are never read: q_map stands in for them
+  const CUtensorMap& km = p.fold ? new_maps[0] : q_map;
+  const CUtensorMap& vm = p.fold ? new_maps[1] : q_map;
+  const cudaError_t e = cudaLaunchKernelEx(&l.cfg, unit_attention_kernel<D>, q_map, kv_map, km, vm, p);
   if (e != cudaSuccess && std::getenv("WS_DEBUG")) {
     cudaFuncAttributes fa{};
     cudaFuncGetAttributes(&fa, unit_attention_kernel<D>);
@@ -687,10 +801,15 @@ int attention_workers(int head_dim) { return use_pair_kernel(head_dim) ? pair_wo
 bool attention_uses_pairs(int head_dim) { return use_pair_kernel(head_dim); }
 
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const CUtensorMap& k_half_map,
-                             const AttnParams& p, int head_dim, int* ctas, cudaStream_t stream) {
-  if (use_pair_kernel(head_dim)) return launch_attention_pair(q_map, k_half_map, kv_map, p, ctas, stream);
-  if (head_dim == 128) return launch_attention_d<128>(q_map, kv_map, p, ctas, stream);
-  if (head_dim == 64) return launch_attention_d<64>(q_map, kv_map, p, ctas, stream);
+                             const CUtensorMap* new_maps, const AttnParams& p, int head_dim, int* ctas,
+                             cudaStream_t stream) {
+  if (p.fold && !new_maps) return cudaErrorInvalidValue;
+  if (use_pair_kernel(head_dim)) {
+    if (p.fold) return cudaErrorInvalidValue;   // the paired kernel reads the cache only
+    return launch_attention_pair(q_map, k_half_map, kv_map, p, ctas, stream);
+  }
+  if (head_dim == 128) return launch_attention_d<128>(q_map, kv_map, new_maps, p, ctas, stream);
+  if (head_dim == 64) return launch_attention_d<64>(q_map, kv_map, new_maps, p, ctas, stream);
   return cudaErrorInvalidValue;
 }
 

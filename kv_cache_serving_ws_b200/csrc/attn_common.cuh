@@ -25,7 +25,7 @@ struct Range {
 struct TileIter {
   int g, len, tiles, gq, qt0, n_units;
   int a, h, j, t, tiles_j, n;
-  int run, run_off, run_row0, run_rows;
+  int run, run_off, run_row0, run_rows, run_new;
   bool first, last;
   __device__ __forceinline__ int qt() const { return qt0 + a; }
   __device__ __forceinline__ int row0() const { return run_row0 + run_off; }
@@ -37,11 +37,14 @@ struct TileIter {
   __device__ __forceinline__ void load_run(const KeyRuns& r) {
     run_row0 = r.row_begin[run];
     run_rows = r.rows[run];
+    run_new = r.from_new[run];
   }
-  // debug builds: the current run lies inside the K/V planes, and so does head h's plane
+  // debug builds: the current run lies inside the K/V planes (or inside k_new / v_new,
+  // whose rows are those of out), and so does head h's plane
   __device__ __forceinline__ void check_run(const AttnParams& p) const {
-    index_ok(run_row0 >= 0 && run_rows > 0 && (int64_t)run_row0 + run_rows <= p.plane_rows && h >= 0 &&
-                 h < p.n_heads && p.plane_k + h < p.planes && p.plane_v + h < p.planes,
+    const int64_t lim = run_new ? p.out_rows : p.plane_rows;
+    index_ok(run_row0 >= 0 && run_rows > 0 && (int64_t)run_row0 + run_rows <= lim && (!run_new || p.fold) &&
+                 h >= 0 && h < p.n_heads && p.plane_k + h < p.planes && p.plane_v + h < p.planes,
              p.status);
   }
   __device__ void init(const Decomp& d, const QueryUnits& u, const KeyRuns& r, const Range& rg) {

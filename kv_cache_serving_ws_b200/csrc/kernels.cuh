@@ -18,11 +18,14 @@ constexpr int kMaxLaneCtas = 1024;
 // Query unit j of a call owns runs [QueryUnits::run_first[j], run_first[j+1]);
 // each run is cut into kBlockN-row tiles, and tile_begin[r] is the first tile
 // of run r among its unit's tiles.
+// A run flagged from_new holds rows of the call's own k_new/v_new ([n_units*Nq][H][D],
+// row_begin counting their token rows) instead of cache rows.
 struct KeyRuns {
   int32_t n_runs;
   int32_t row_begin[kMaxRuns];
   int32_t rows[kMaxRuns];
   int32_t tile_begin[kMaxRuns];
+  int8_t from_new[kMaxRuns];
 };
 
 // The query units of one call (one for the per-unit step, several for a
@@ -127,6 +130,14 @@ struct AttnParams {
   int64_t fix_slots;        // merge counters behind fix_count
   int64_t plane_rows;       // rows of each K/V plane
   int64_t planes;           // planes of the K/V maps
+  // The call's own latent K/V.  fold = 1: the kernel reads those key rows from k_new /
+  // v_new (runs flagged from_new) and writes them into their cache rows itself; fold =
+  // 0: they were written into the cache before the launch.
+  int32_t fold;
+  const uint16_t* k_new;    // [n_units * Nq][H][D] bf16
+  const uint16_t* v_new;
+  uint16_t* cache;          // the K/V planes [planes][plane_rows][D]
+  int64_t latent_row0[kMaxQUnits];  // plane row of query unit j's first latent row
   Decomp dec;
   QueryUnits qu;
   KeyRuns runs;
@@ -147,8 +158,11 @@ int encode_q_map(CUtensorMap* map, const void* q, int head_dim, int n_heads, int
 // (attention_pair.cu) where the device can hold its clusters.  `kv_map` has
 // whole-tile boxes, `k_half_map` boxes of 64 rows.  `p.dec` must come from
 // decompose() with attention_workers(head_dim) workers.
+// With p.fold = 1, new_maps[0] and new_maps[1] map k_new and v_new like q_map (the
+// single-SM kernel only; the paired kernel takes p.fold = 0).
 cudaError_t launch_attention(const CUtensorMap& q_map, const CUtensorMap& kv_map, const CUtensorMap& k_half_map,
-                             const AttnParams& p, int head_dim, int* ctas, cudaStream_t stream);
+                             const CUtensorMap* new_maps, const AttnParams& p, int head_dim, int* ctas,
+                             cudaStream_t stream);
 // Workers (CTAs, or CTA pairs) of the kernel launch_attention uses for head_dim.
 int attention_workers(int head_dim);
 bool attention_uses_pairs(int head_dim);

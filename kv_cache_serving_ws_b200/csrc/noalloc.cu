@@ -184,7 +184,8 @@ int noalloc_impl(const uint16_t* q, const uint16_t* kv, uint16_t* out, int32_t n
   // the status word and the merge counters start at zero (a call that gave up may have left them set)
   if (cudaMemsetAsync(p.status, 0, kStatusBytes + fix_bytes, stream) != cudaSuccess) return WS_ERR_CUDA;
   p.fixup = use_fixup(p.dec) ? 1 : 0;
-  if (launch_attention(q_map, kv_map, k_half_map, p, head_dim, nullptr, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (launch_attention(q_map, kv_map, k_half_map, nullptr, p, head_dim, nullptr, stream) != cudaSuccess)
+    return WS_ERR_CUDA;
   bool any_split = false;
   for (int qt = 0; qt < n_qtiles && !any_split && !p.fixup; ++qt)
     for (int h = 0; h < n_heads && !any_split; ++h) {

@@ -77,7 +77,7 @@ int resident(const ws_cache* h, int session, int64_t unit) {
 }
 
 int plan_runs(const ws_cache_config& cfg, const int64_t* slot_unit, const uint8_t* latent_ready, int layer,
-              int64_t unit, int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs) {
+              int64_t unit, int64_t new_from, int32_t* row_begin, int32_t* rows, int32_t max_runs, int32_t* n_runs) {
   const int C = cfg.history_units + 1;
   const int Nq = cfg.n_video + cfg.n_audio;
   const int T = cfg.n_cond + Nq;
@@ -87,7 +87,8 @@ int plan_runs(const ws_cache_config& cfg, const int64_t* slot_unit, const uint8_
   for (int s = 0; s < C; ++s) {
     const int64_t u = slot_unit[s];
     if (u < 0 || u < lo || u > unit) continue;
-    const bool lat = (u == unit) || latent_ready[(size_t)s * cfg.n_layers + layer];
+    // units from new_from on are the call's own: their latent rows come from k_new / v_new
+    const bool lat = (new_from < 0 || u < new_from) && ((u == unit) || latent_ready[(size_t)s * cfg.n_layers + layer]);
     const int64_t b = (int64_t)s * T;
     const int64_t e = b + cfg.n_cond + (lat ? Nq : 0);
     if (e == b) continue;
@@ -173,22 +174,47 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
     if (rd.empty()) rd = h->rings[(size_t)sessions[j]].latent_ready;
     rd[(size_t)(units[j] % h->C) * L + layer] = 1;
   }
+  // The single-SM kernel writes the call's latent K/V itself and reads those key rows
+  // from k_new / v_new (no separate write launch) when every session has one query
+  // unit in the call.  In a prefill stretch the cache interleaves each unit's
+  // conditioning rows with its latent rows, so reading the latents elsewhere would cut
+  // the key runs into short tiles: those calls, and the paired kernel, write first and
+  // read the cache.
+  bool fold = !attention_uses_pairs(D);
+  for (int j = 1; j < n; ++j)
+    if (sessions[j] == sessions[j - 1]) fold = false;
   AttnParams p{};
   p.qu.n_units = n;
   p.qu.rows = h->Nq;
   int runs = 0, tiles = 0;
   int64_t keys = 0;
+  int j_first = 0;   // first query unit of the current session's stretch
   for (int j = 0; j < n; ++j) {
+    if (j > 0 && sessions[j] != sessions[j - 1]) j_first = j;
     p.qu.run_first[j] = runs;
     p.qu.tile_start[j] = tiles;
     int32_t nr = 0;
     const int sess = sessions[j];
+    const int64_t u_first = units[j_first];
     const int st = plan_runs(h->cfg, h->rings[(size_t)sess].slot_unit.data(), ready[(size_t)sess].data(), layer,
-                             units[j], p.runs.row_begin + runs, p.runs.rows + runs, kMaxRuns - runs, &nr);
+                             units[j], fold ? u_first : -1, p.runs.row_begin + runs, p.runs.rows + runs,
+                             kMaxRuns - runs, &nr);
     if (st != WS_OK) return st;
-    int t = 0;
     for (int r = runs; r < runs + nr; ++r) {
       p.runs.row_begin[r] += (int32_t)(sess * h->session_rows);
+      p.runs.from_new[r] = 0;
+    }
+    if (fold) {
+      // the visible units of the stretch, u_lo .. units[j]: consecutive token rows of k_new
+      const int64_t u_lo = std::max<int64_t>(u_first, units[j] - U);
+      if (runs + nr == kMaxRuns) return WS_ERR_UNSUPPORTED;
+      p.runs.row_begin[runs + nr] = (int32_t)((j_first + (u_lo - u_first)) * h->Nq);
+      p.runs.rows[runs + nr] = (int32_t)((units[j] - u_lo + 1) * h->Nq);
+      p.runs.from_new[runs + nr] = 1;
+      ++nr;
+    }
+    int t = 0;
+    for (int r = runs; r < runs + nr; ++r) {
       p.runs.tile_begin[r] = t;
       t += (p.runs.rows[r] + kBlockN - 1) / kBlockN;
       keys += p.runs.rows[r];
@@ -219,10 +245,25 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   CUtensorMap q_map;
   if (encode_q_map(&q_map, q, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
 
-  // 1. the query units' latent K/V of this layer into their slots
+  // 1. the query units' latent K/V of this layer into their slots: inside the
+  //    attention launch (fold), else by one write launch per unit
   const size_t unit_elems = (size_t)h->Nq * H * D;
+  CUtensorMap new_maps[2];
+  if (fold) {
+    if (encode_q_map(&new_maps[0], k_new, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
+    if (encode_q_map(&new_maps[1], v_new, D, H, n * h->Nq) != 0) return WS_ERR_CUDA;
+    p.fold = 1;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.cache = h->kv;
+  }
   for (int j = 0; j < n; ++j) {
     const size_t slot = (size_t)(units[j] % h->C);
+    p.latent_row0[j] = sessions[j] * h->session_rows + (int64_t)slot * h->T + h->cfg.n_cond;
+    if (fold) {
+      h->rings[(size_t)sessions[j]].latent_ready[slot * L + layer] = 1;
+      continue;
+    }
     AppendParams a{};
     a.src_k = k_new + j * unit_elems;
     a.src_v = v_new + j * unit_elems;
@@ -263,7 +304,9 @@ int attention_impl(ws_cache* h, int layer, const int32_t* sessions, const int64_
   cudaEvent_t* ev = h->profiling && !h->capturing ? h->ev_attn.next() : nullptr;
   if (ev) cudaEventRecord(ev[0], stream);
   int ctas = 0;
-  if (launch_attention(q_map, h->kv_map, h->k_half_map, p, D, &ctas, stream) != cudaSuccess) return WS_ERR_CUDA;
+  if (launch_attention(q_map, h->kv_map, h->k_half_map, fold ? new_maps : nullptr, p, D, &ctas, stream) !=
+      cudaSuccess)
+    return WS_ERR_CUDA;
   if (ev) cudaEventRecord(ev[1], stream);
   if (any_split) {
     ev = h->profiling && !h->capturing ? h->ev_comb.next() : nullptr;
@@ -358,7 +401,7 @@ int ws_plan_visible(const ws_cache_config* cfg, const int64_t* slot_unit, const 
   if (!config_ok(cfg) || !slot_unit || !latent_ready || !row_begin || !rows || !n_runs || max_runs < 0)
     return WS_ERR_ARG;
   if (layer < 0 || layer >= cfg->n_layers || unit < 0) return WS_ERR_ARG;
-  return plan_runs(*cfg, slot_unit, latent_ready, layer, unit, row_begin, rows, max_runs, n_runs);
+  return plan_runs(*cfg, slot_unit, latent_ready, layer, unit, -1, row_begin, rows, max_runs, n_runs);
 }
 
 int ws_pool_create(ws_cache_t** out, const ws_cache_config* cfg, int32_t n_sessions, cudaStream_t stream) {

@@ -11,7 +11,7 @@ sys.path.insert(0, HERE)
 
 import numpy as np  # noqa: E402
 
-from gpu_util import ATOL_MAX, ATOL_MEAN  # noqa: E402
+from gpu_util import ATOL_MAX, ATOL_MEAN, STRESSED_MAX, STRESSED_MEAN, half_ulp_bf16  # noqa: E402
 from kv_cache_serving_ws_b200 import native as ws  # noqa: E402
 from oracle import ws_oracle as orc  # noqa: E402
 from test_gpu_attention import Pair, _times4  # noqa: E402
@@ -29,7 +29,8 @@ def run(name, cfg, units, commit_skip=(), splits=0, layer=0, qs=None, tol=(ATOL_
     kernel = ws.ws_profile_read(p.h)["last_kernel"]
     p.close()
     d = np.abs(got - want)
-    ok = kernel == 2 and np.all(np.isfinite(got)) and d.max() <= tol[0] and d.mean() <= tol[1]
+    bound = tol[0] + (half_ulp_bf16(want) if tol[0] > ATOL_MAX else 0.0)   # stressed: plus the output's rounding
+    ok = kernel == 2 and np.all(np.isfinite(got)) and np.all(d <= bound) and d.mean() <= tol[1]
     print(f"{name}: kernel={kernel} max={d.max():.2e} mean={d.mean():.2e} {'ok' if ok else 'FAIL'}", flush=True)
     if not ok:
         sys.exit(1)
@@ -63,7 +64,7 @@ if __name__ == "__main__":
     run("same, 4 pairs per lane", C(2, 3, 128, 130, 3, 5, 4), [0, 1, 2, 4, 5, 6], commit_skip=(5,), splits=4,
         layer=1)
     run("stressed query (x4)", C(2, 3, 128, 130, 3, 5, 4), [0, 1, 2, 4, 5, 6], commit_skip=(5,), splits=1,
-        qs=_times4, tol=(2e-2, 2e-3))
+        qs=_times4, tol=(STRESSED_MAX, STRESSED_MEAN))
     run("two query blocks, 8 heads, all pairs", C(1, 8, 128, 300, 4, 32, 6), list(range(7)))
     run("long items merged inside the kernel", C(1, 1, 128, 250, 6, 0, 511), list(range(512)), splits=12)
     poisoned_neighbour_rows()

@@ -143,3 +143,28 @@ def test_argument_errors_leave_state_unchanged():
     assert info["cache_bytes"] == 1 * 2 * 2 * 2 * 6 * 64 * 2
     assert ws.ws_sync(t.h, check=False) == ws.WS_OK
     t.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("head_dim", [64, 128])
+def test_latent_write_inside_the_attention_launch(head_dim):
+    """The single-SM kernel writes the call's latent K/V itself: one launch per call
+    (no separate write), and the written rows equal k_new / v_new bit for bit, over
+    a ragged unit (Nq = 133) with the ring wrapped."""
+    require_gpu()
+    cfg = orc.Config(n_layers=2, n_heads=3, head_dim=head_dim, n_video=130, n_audio=3, n_cond=5, history_units=2)
+    t = Twin(cfg)
+    for u in range(6):
+        t.append(u, orc.SEG_COND)
+        if u < 5:
+            t.append(u, orc.SEG_LATENT)
+    ws.ws_profile_enable(t.h, True)
+    t.attention(1, 5)
+    t.attention(0, 5)
+    torch.cuda.synchronize()
+    prof = ws.ws_profile_read(t.h)
+    ws.ws_profile_enable(t.h, False)
+    assert prof["last_kernel"] == 1
+    assert prof["latent_write_launches"] == 0 and prof["attention_launches"] == 2
+    t.check_state()
+    t.close()
