@@ -371,15 +371,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_o(tmem, a);
         const uint32_t p_tmem = tmem_s(tmem, a);
-        const int steps = (valid + 15) >> 4;
-#pragma unroll
-        for (int kk = 0; kk < kBlockN / 16; ++kk) {
-          if (kk >= steps) break;
-          // 16 keys = 8 TMEM columns; V: 16 rows of 128 bytes, the next 64
-          // head-dim columns one chunk (kBlockN rows) further
+        // 16 keys = 8 TMEM columns; V: 16 rows of 128 bytes, the next 64 head-dim
+        // columns one chunk (kBlockN rows) further
+        auto pv_step = [&](int kk) {
           const uint64_t db = umma_smem_desc_sw128(v_base + s * S::kTileBytes + kk * 16 * kRowBytes,
                                                    kBlockN * kRowBytes, 1024);
           if (elect_one()) umma_bf16_ts(o_tmem, p_tmem + (uint32_t)(kk * 8), db, idesc_o, (!it.first || kk > 0) ? 1u : 0u);
+        };
+        if (valid == kBlockN) {
+          // whole tile (all but a run's last): the 8 steps with no per-step test
+#pragma unroll
+          for (int kk = 0; kk < kBlockN / 16; ++kk) pv_step(kk);
+        } else {
+          // a run's last tile: stop after the 16-key step holding its last valid row
+          const int steps = (valid + 15) >> 4;
+#pragma unroll 1
+          for (int kk = 0; kk < steps; ++kk) pv_step(kk);
         }
         if (it.last && elect_one()) umma_commit(&bars[kOFull + a]);
         if (a == kQTiles - 1 && elect_one()) umma_commit(&bars[kVEmpty + s]);
