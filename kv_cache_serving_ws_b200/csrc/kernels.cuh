@@ -241,6 +241,9 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
+// A launch recorded into a CUDA graph (stream capture) goes without the attribute:
+// with programmatic edges in it, updating the unit program's executable graph in
+// place made the host wait for the previous unit's execution.
 struct PdlLaunch {
   cudaLaunchConfig_t cfg{};
   cudaLaunchAttribute attr[1];
@@ -252,7 +255,12 @@ struct PdlLaunch {
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) {
+      cudaGetLastError();
+      cs = cudaStreamCaptureStatusActive;
+    }
+    cfg.numAttrs = cs == cudaStreamCaptureStatusNone ? 1 : 0;
   }
 };
 
