@@ -90,6 +90,16 @@ def test_noalloc_matches_unit_attention_on_two_calls_in_a_row():
         heads = [0, H - 1]
         d = np.abs(got[:, heads] - _oracle_heads(q, kv, heads))
         assert d.max() <= ATOL_MAX and d.mean() <= ATOL_MEAN, (cfg, float(d.max()), float(d.mean()))
+    # the entry point allocates no device memory: after the calls above (module and
+    # scratch already loaded), more calls leave the device's free memory as it was
+    # (any cudaMalloc takes at least a 2 MiB page)
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    for _ in range(3):
+        assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, check=False) == ws.WS_OK
+    torch.cuda.synchronize()
+    assert ws.ws_attention_noalloc_sync(check=False) == ws.WS_OK
+    assert free0 - torch.cuda.mem_get_info()[0] < (1 << 20)
 
 
 @pytest.mark.gpu
