@@ -131,8 +131,9 @@ int ws_cache_append(ws_cache_t* h, int64_t unit, int seg,
  * this layer if they have been written (by this call for u' = unit, by an
  * earlier commit or attention call otherwise).  Within a unit the attention is
  * bidirectional (video and audio together); across units it is causal.
- * The write and the attention are one kernel launch (the unit's own key tiles
- * are read from k_new / v_new directly); q, k_new and v_new are read, like every
+ * With the default kernel the write and the attention are one kernel launch
+ * (the unit's own key tiles are read from k_new / v_new directly; the opt-in
+ * paired kernel writes first).  q, k_new and v_new are read, like every
  * buffer argument, by work queued on `stream`, so they must stay unchanged until
  * that work has run.
  * out: [Nq][H][D] bf16 (written, not accumulated).  Arithmetic: bf16 tensor-core
