@@ -151,3 +151,28 @@ def test_noalloc_rejects_bad_arguments_before_any_launch():
         with torch.cuda.device(1):
             other = torch.cuda.Stream()
         assert ws.ws_attention_noalloc(t, t, t, 1, 1, 1, 64, stream=other, check=False) == ws.WS_ERR_ARG
+
+
+@pytest.mark.gpu
+def test_noalloc_on_a_second_device_after_the_first():
+    """Kernel attributes (the shared-memory opt-in) and the scratch address are kept per
+    device: a call on device 1 after calls on device 0 gives the same bytes.  Needs two
+    GPUs; skipped otherwise."""
+    require_gpu()
+    if torch.cuda.device_count() < 2:
+        pytest.skip("one GPU visible")
+    H, D, Nq, Nk = 3, 128, 260, 700
+    key = lambda kind: synth.stream_key(31, kind, 0, 0)
+    outs = []
+    for dev in (0, 1):
+        with torch.cuda.device(dev):
+            q = torch.empty((Nq, H, D), dtype=torch.bfloat16, device=f"cuda:{dev}")
+            kv = torch.empty((2, H, Nk, D), dtype=torch.bfloat16, device=f"cuda:{dev}")
+            ws.synth_fill(q, key(synth.KIND_Q))
+            ws.synth_fill(kv, key(synth.KIND_K_NEW))
+            out = torch.empty_like(q)
+            stream = torch.cuda.current_stream()
+            assert ws.ws_attention_noalloc(q, kv, out, Nq, Nk, H, D, stream=stream, check=False) == ws.WS_OK
+            assert ws.ws_attention_noalloc_sync(stream=stream, check=False) == ws.WS_OK
+            outs.append(out.cpu())
+    assert torch.equal(outs[0], outs[1])
